@@ -1,0 +1,179 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention (KDA) core library, libkda.so.
+ *
+ * KDA is a gated delta-rule linear attention with a channel-wise forget gate.
+ * Per (sequence, head) it keeps a dk x dv fp32 state S (row = key channel) and,
+ * token by token,
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp g_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = scale * S_t^T q_t                      (scale = 1/sqrt(dk) by default)
+ *     y_t = o_t / sqrt(mean_j o_t[j]^2 + eps) * w * sigmoid(gate_t)   (when gate != NULL)
+ *
+ * Sources of each part:
+ *   - delta rule on the generalised Householder transformation, chunkwise
+ *     ("piecewise parallel") form: "Kimi K3 from Moonshot AI: 2.8 Trillion
+ *     Parameters Unveiled", section "Kimi Delta Attention (KDA)";
+ *   - fixed-size state, constant per-token decode cost, per-channel forgetting,
+ *     head-wise RMSNorm followed by an input-dependent output gate, bounded
+ *     log-decay that lets every causal tile be a dense tensor-core product:
+ *     "Kimi K3 Architecture Explained: KDA, Attention Residuals and LatentMoE",
+ *     section "Token mixing: what KDA is and why 3:1";
+ *   - g_min = -5, so a 16-token tile's cumulative log-decay lies in (-80, 0) and
+ *     its reciprocal factors (<= e^80) fit the BF16 range: "Kimi K3: Engineering a
+ *     2.8 Trillion Parameter Frontier", section "Dimension 1: Sequence Length via
+ *     Hybrid KDA-Gated MLA".
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, row-major and
+ *     contiguous, 16-byte aligned.  Exceptions are marked HOST.
+ *   - The library allocates no memory, never synchronises the stream (except
+ *     kda_read_device_error) and launches its kernels on the given cudaStream_t
+ *     (passed as void*; NULL = the legacy default stream).
+ *   - Host-detectable errors (NULL pointers, shapes, alignment, dtype, workspace
+ *     size) return before anything is launched.  A failed launch returns
+ *     KDA_ERR_CUDA.  Errors found on the device (a decay outside [g_min, 0] or a
+ *     bad state index in checked mode, a bounded wait that ran out) are written to a
+ *     device error word and read back with kda_read_device_error.
+ *   - Precondition: every g lies in [KDA_G_MIN, 0].  Without KDA_FLAG_CHECK_DECAY a
+ *     value below KDA_G_MIN is undefined behaviour for the bf16 tensor-core path
+ *     (its tile factors may overflow); with the flag the kernel reports
+ *     KDA_ERR_DECAY_OUT_OF_RANGE in the error word.
+ *   - Outputs must not alias inputs.  Decode updates `state` in place by design.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KDA_VERSION_MAJOR 0
+#define KDA_VERSION_MINOR 1
+
+/* Lower bound of the per-token log-decay (scaled-sigmoid floor). */
+#define KDA_G_MIN (-5.0f)
+
+typedef enum kda_status {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARGUMENT = 1,   /* NULL pointer, bad shape, misaligned pointer, bad cu_seqlens */
+  KDA_ERR_UNSUPPORTED = 2,        /* valid request this build does not implement (e.g. dk = 96) */
+  KDA_ERR_WORKSPACE_TOO_SMALL = 3,
+  KDA_ERR_CUDA = 4,               /* a CUDA runtime call or kernel launch failed */
+  KDA_ERR_TIMEOUT = 5,            /* (device) a bounded wait inside a kernel ran out */
+  KDA_ERR_DECAY_OUT_OF_RANGE = 6, /* (device, checked mode) some g outside [KDA_G_MIN, 0] */
+  KDA_ERR_BAD_STATE_INDEX = 7     /* (device, checked mode) state_indices[n] outside [0, num_slots) */
+} kda_status;
+
+typedef enum kda_dtype {
+  KDA_BF16 = 0, /* q, k, v, g, beta, gate and out in bfloat16 */
+  KDA_F32 = 1   /* the same tensors in float32 */
+} kda_dtype;
+
+/* flags (bitwise OR) */
+#define KDA_FLAG_CHECK_DECAY 0x1u      /* verify g in [KDA_G_MIN, 0] (and state indices) on the device */
+#define KDA_FLAG_FORCE_SIMT 0x2u       /* prefill: use the fp32 CUDA-core chunk kernel even for bf16 */
+#define KDA_FLAG_TEST_FORCE_TIMEOUT 0x4u /* tests only: bounded waits give up at once -> KDA_ERR_TIMEOUT */
+
+/* ------------------------------------------------------------------------------------------
+ * Chunkwise prefill.
+ *
+ * Shapes (T_tot = total_tokens, N = num_seqs):
+ *   q, k, g       [T_tot, H, dk]   dtype
+ *   v, gate       [T_tot, H, dv]   dtype   (gate = gate logits; NULL => no RMSNorm/gate
+ *                                            epilogue, out = raw scale * S^T q)
+ *   beta          [T_tot, H]       dtype
+ *   norm_weight   [dv]             float32 or NULL (= all ones)
+ *   initial_state [N, H, dk, dv]   float32 or NULL (= zeros)
+ *   out           [T_tot, H, dv]   dtype
+ *   final_state   [N, H, dk, dv]   float32 or NULL (not written)
+ *   cu_seqlens    HOST int32 [N + 1]: sequence n is tokens [cu_seqlens[n], cu_seqlens[n+1]);
+ *                 cu_seqlens[0] = 0, non-decreasing, cu_seqlens[N] = T_tot (zero-length
+ *                 sequences are allowed: their final state is their initial state).
+ *                 NULL => N sequences of T_tot / N tokens each (a dense [N, T, H, d] batch).
+ *   dk, dv in {64, 128}.  bf16 with dk = dv = 128 runs the tcgen05 tensor-core kernel;
+ *   every other combination (and KDA_FLAG_FORCE_SIMT) runs the fp32 CUDA-core kernel.
+ *   split_segments: 0 = automatic; 1 = never split a sequence; P > 1 = split every
+ *   sequence into P segments processed in parallel (state carried by a combine pass).
+ *   workspace: device scratch of at least kda_chunk_fwd_workspace_size() bytes, 256-byte
+ *   aligned, owned by the caller, not shared by calls that may overlap on the GPU.  Its
+ *   first 4 bytes are the device error word, cleared at the start of every call.
+ * ------------------------------------------------------------------------------------------ */
+typedef struct kda_chunk_args {
+  int32_t num_seqs;
+  int64_t total_tokens;
+  const int32_t* cu_seqlens; /* HOST */
+  int32_t H, dk, dv;
+  kda_dtype dtype;
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* g;
+  const void* beta;
+  const void* gate;
+  const float* norm_weight;
+  const float* initial_state;
+  void* out;
+  float* final_state;
+  float scale; /* 0 => 1/sqrt(dk) */
+  float eps;   /* RMSNorm epsilon inside the square root (1e-6 in the reference configs) */
+  uint32_t flags;
+  int32_t split_segments;
+  void* workspace;
+  size_t workspace_bytes;
+} kda_chunk_args;
+
+/* Bytes of workspace kda_chunk_fwd needs for these arguments (pure host computation). */
+kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args* args, size_t* bytes);
+
+/* Launch the chunkwise prefill on `cuda_stream`.  Asynchronous. */
+kda_status kda_chunk_fwd(const kda_chunk_args* args, void* cuda_stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Decode step: one new token for each of N sequences, states updated in place.
+ *
+ *   q, k, g       [N, H, dk]  dtype;  v, gate [N, H, dv] dtype (gate NULL => no epilogue)
+ *   beta          [N, H]      dtype
+ *   state         [num_slots, H, dk, dv] float32, read and written in place
+ *   state_indices [N] int32 device pointer (sequence n uses slot state_indices[n]) or NULL
+ *                 (slot n; then num_slots >= N).  Slots used by two sequences race.
+ *   out           [N, H, dv]  dtype
+ *   error_word    device uint32 or NULL.  Sticky: kernels only set it; the caller zeroes it
+ *                 before first use and kda_read_device_error zeroes it after reading.
+ * ------------------------------------------------------------------------------------------ */
+typedef struct kda_decode_args {
+  int32_t N, H, dk, dv;
+  kda_dtype dtype;
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* g;
+  const void* beta;
+  const void* gate;
+  const float* norm_weight;
+  float* state;
+  int32_t num_slots;
+  const int32_t* state_indices;
+  void* out;
+  float scale; /* 0 => 1/sqrt(dk) */
+  float eps;
+  uint32_t flags;
+  uint32_t* error_word;
+} kda_decode_args;
+
+kda_status kda_decode_step(const kda_decode_args* args, void* cuda_stream);
+
+/* Synchronise `cuda_stream`, read the device error word (a kda_chunk_fwd workspace or a
+ * decode error_word), reset it to zero and return the status it held (KDA_OK if none).
+ * Returns KDA_ERR_CUDA if the synchronisation or the copy fails. */
+kda_status kda_read_device_error(const void* error_word, void* cuda_stream);
+
+/* Static, NUL-terminated name of a status code. */
+const char* kda_status_string(kda_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KDA_H */

@@ -1,0 +1,269 @@
+// kda_api.cu -- the C ABI of libkda: argument validation, work planning and dispatch.
+//
+// Host-side only (no kernels here).  Every check that can fail on the host runs before
+// the first CUDA call, so a rejected call has no side effect on the device.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+#include <vector>
+
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+// Number of SMs the automatic sequence split plans for (B200: 148).  A constant, so that
+// kda_chunk_fwd_workspace_size and kda_chunk_fwd agree without querying a device.
+constexpr int kPlanSMs = 148;
+constexpr int kSegAlign = 64;     // segment lengths are multiples of the largest chunk
+constexpr int kMinAutoSeg = 2048; // automatic split: tokens per segment at least this
+constexpr size_t kErrBytes = 256;
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+struct SeqSpan {
+  int32_t tok0, len, seq;
+};
+
+struct Layout {
+  std::vector<SeqSpan> seqs;   // every sequence
+  std::vector<int32_t> nseg;   // segments per sequence (1 = not split)
+  std::vector<int32_t> seglen; // segment length per sequence
+  std::vector<int32_t> slot0;  // first workspace slot of a split sequence
+  int32_t slots = 0;
+  bool any_split = false;
+};
+
+kda_status validate(const kda_chunk_args* a) {
+  if (!a) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->num_seqs < 0 || a->total_tokens < 0 || a->H <= 0) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->total_tokens > INT32_MAX) return KDA_ERR_UNSUPPORTED;
+  if (a->dtype != KDA_BF16 && a->dtype != KDA_F32) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->dk <= 0 || a->dv <= 0) return KDA_ERR_INVALID_ARGUMENT;
+  if ((a->dk != 64 && a->dk != 128) || (a->dv != 64 && a->dv != 128)) return KDA_ERR_UNSUPPORTED;
+  if (a->split_segments < 0) return KDA_ERR_INVALID_ARGUMENT;
+  if (!(a->eps >= 0.f) || !(a->scale >= 0.f)) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->num_seqs == 0 && a->total_tokens != 0) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->total_tokens > 0) {
+    const void* req[] = {a->q, a->k, a->v, a->g, a->beta, a->out};
+    for (const void* p : req)
+      if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+    if (a->gate && !aligned16(a->gate)) return KDA_ERR_INVALID_ARGUMENT;
+  }
+  if (a->norm_weight && !aligned16(a->norm_weight)) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->initial_state && !aligned16(a->initial_state)) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->final_state && !aligned16(a->final_state)) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->cu_seqlens) {
+    if (a->cu_seqlens[0] != 0) return KDA_ERR_INVALID_ARGUMENT;
+    for (int32_t n = 0; n < a->num_seqs; ++n)
+      if (a->cu_seqlens[n + 1] < a->cu_seqlens[n]) return KDA_ERR_INVALID_ARGUMENT;
+    if ((int64_t)a->cu_seqlens[a->num_seqs] != a->total_tokens) return KDA_ERR_INVALID_ARGUMENT;
+  } else if (a->num_seqs > 0 && a->total_tokens % a->num_seqs != 0) {
+    return KDA_ERR_INVALID_ARGUMENT;
+  }
+  return KDA_OK;
+}
+
+int32_t round_up(int64_t x, int32_t m) { return (int32_t)(((x + m - 1) / m) * m); }
+
+Layout make_layout(const kda_chunk_args* a) {
+  Layout L;
+  const int32_t N = a->num_seqs;
+  L.seqs.resize(N);
+  for (int32_t n = 0; n < N; ++n) {
+    int32_t t0, len;
+    if (a->cu_seqlens) {
+      t0 = a->cu_seqlens[n];
+      len = a->cu_seqlens[n + 1] - a->cu_seqlens[n];
+    } else {
+      len = (int32_t)(a->total_tokens / N);
+      t0 = n * len;
+    }
+    L.seqs[n] = {t0, len, n};
+  }
+  // Sequence split: automatic when the (sequence, head) units cannot fill half the GPU.
+  int64_t busy = 0;
+  for (const auto& s : L.seqs) busy += (s.len > 0) ? a->H : 0;
+  int32_t P = 1;
+  bool auto_mode = a->split_segments == 0;
+  if (auto_mode) {
+    if (busy > 0 && busy * 2 <= kPlanSMs) P = (int32_t)std::min<int64_t>(64, kPlanSMs / busy);
+  } else {
+    P = a->split_segments;
+  }
+  L.nseg.assign(N, 1);
+  L.seglen.assign(N, 0);
+  L.slot0.assign(N, -1);
+  for (int32_t n = 0; n < N; ++n) {
+    const int32_t len = L.seqs[n].len;
+    L.seglen[n] = len;
+    if (P <= 1 || len <= kSegAlign) continue;
+    int32_t p = P;
+    if (auto_mode) p = (int32_t)std::min<int64_t>(p, len / kMinAutoSeg);
+    if (p <= 1) continue;
+    const int32_t sl = round_up((len + p - 1) / p, kSegAlign);
+    const int32_t np = (len + sl - 1) / sl;
+    if (np <= 1) continue;
+    L.nseg[n] = np;
+    L.seglen[n] = sl;
+    L.slot0[n] = L.slots;
+    L.slots += np;
+    L.any_split = true;
+  }
+  return L;
+}
+
+size_t workspace_bytes(const kda_chunk_args* a, const Layout& L) {
+  size_t b = kErrBytes;
+  if (L.slots > 0) {
+    const size_t per = (size_t)a->dk * a->dv + (size_t)a->dk * (a->dv + a->dk);
+    b += (size_t)L.slots * a->H * per * sizeof(float);
+  }
+  return b;
+}
+
+// Launch `segs` (all of one role class) in batches of kPlanMax, longest first.
+cudaError_t run_segments(std::vector<Seg>& segs, const ChunkParams& p, kda_dtype dtype, bool use_tc,
+                         cudaStream_t stream) {
+  std::stable_sort(segs.begin(), segs.end(), [](const Seg& x, const Seg& y) { return x.len > y.len; });
+  static thread_local Plan plan;  // 24 KB: kept off the stack
+  for (size_t b = 0; b < segs.size(); b += kPlanMax) {
+    const size_t n = std::min<size_t>(kPlanMax, segs.size() - b);
+    plan.n_seg = (int32_t)n;
+    plan.H = p.H;
+    for (size_t i = 0; i < n; ++i) plan.seg[i] = segs[b + i];
+    cudaError_t e = use_tc ? launch_chunk_tc(plan, p, stream) : launch_chunk_simt(plan, p, dtype, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args* a, size_t* bytes) {
+  if (!bytes) return KDA_ERR_INVALID_ARGUMENT;
+  kda_status s = validate(a);
+  if (s != KDA_OK) return s;
+  *bytes = workspace_bytes(a, make_layout(a));
+  return KDA_OK;
+}
+
+extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) {
+  kda_status s = validate(a);
+  if (s != KDA_OK) return s;
+  const Layout L = make_layout(a);
+  if (!a->workspace || ((uintptr_t)a->workspace & 255u) != 0) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->workspace_bytes < workspace_bytes(a, L)) return KDA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t stream = (cudaStream_t)cuda_stream;
+
+  ChunkParams p;
+  p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta; p.gate = a->gate;
+  p.norm_weight = a->norm_weight;
+  p.initial_state = a->initial_state;
+  p.out = a->out;
+  p.final_state = a->final_state;
+  p.error_word = (uint32_t*)a->workspace;
+  float* ws = (float*)((char*)a->workspace + kErrBytes);
+  p.ws_state = L.slots ? ws : nullptr;
+  p.ws_local = L.slots ? ws + (size_t)L.slots * a->H * a->dk * a->dv : nullptr;
+  p.H = a->H; p.dk = a->dk; p.dv = a->dv;
+  p.scale = a->scale > 0.f ? a->scale : 1.0f / sqrtf((float)a->dk);
+  p.eps = a->eps;
+  p.flags = a->flags;
+
+  if (cudaMemsetAsync(a->workspace, 0, sizeof(uint32_t), stream) != cudaSuccess) return KDA_ERR_CUDA;
+  if (a->num_seqs == 0) return KDA_OK;
+
+  const bool use_tc = false;
+
+  // Pass 1 of split sequences: the head segment from the true initial state, and the
+  // other non-final segments from [0 | I] (local state and transition matrix).
+  std::vector<Seg> head, local, whole;
+  for (int32_t n = 0; n < a->num_seqs; ++n) {
+    const SeqSpan& sp = L.seqs[n];
+    const int32_t np = L.nseg[n];
+    if (np == 1) {
+      whole.push_back({sp.tok0, sp.len, sp.seq, kRoleWhole, -1, 1});
+      continue;
+    }
+    const int32_t sl = L.seglen[n], b = L.slot0[n];
+    for (int32_t q = 0; q < np; ++q) {
+      const int32_t t0 = sp.tok0 + q * sl;
+      const int32_t len = std::min(sl, sp.len - q * sl);
+      if (q == 0) head.push_back({t0, len, sp.seq, kRoleHead, b, 0});
+      else if (q < np - 1) local.push_back({t0, len, sp.seq, kRoleLocal, b + q, 0});
+      if (q == 0) whole.push_back({t0, len, sp.seq, kRoleWhole, b, 0});
+      else whole.push_back({t0, len, sp.seq, kRoleFromWs, b + q, q == np - 1 ? 1 : 0});
+    }
+  }
+  cudaError_t e = cudaSuccess;
+  if (!head.empty()) e = run_segments(head, p, a->dtype, false, stream);
+  if (e == cudaSuccess && !local.empty()) e = run_segments(local, p, a->dtype, false, stream);
+  if (e == cudaSuccess && L.any_split) {
+    // combine: S_start(q+1) = M_q S_start(q) + S_loc(q), sequential over q per (sequence, head)
+    static thread_local Plan plan;
+    plan.H = a->H;
+    plan.n_seg = 0;
+    for (int32_t n = 0; n < a->num_seqs && e == cudaSuccess; ++n) {
+      if (L.nseg[n] <= 2) continue;
+      plan.seg[plan.n_seg++] = {L.seqs[n].tok0, L.nseg[n], L.seqs[n].seq, kRoleLocal, L.slot0[n], 0};
+      if (plan.n_seg == kPlanMax) {
+        e = launch_split_combine(plan, p, 0, stream);
+        plan.n_seg = 0;
+      }
+    }
+    if (e == cudaSuccess && plan.n_seg > 0) e = launch_split_combine(plan, p, 0, stream);
+  }
+  if (e == cudaSuccess) e = run_segments(whole, p, a->dtype, use_tc, stream);
+  return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" kda_status kda_decode_step(const kda_decode_args* a, void* cuda_stream) {
+  if (!a) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->N < 0 || a->H <= 0 || a->num_slots < 0) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->dtype != KDA_BF16 && a->dtype != KDA_F32) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->dk <= 0 || a->dv <= 0) return KDA_ERR_INVALID_ARGUMENT;
+  if ((a->dk != 64 && a->dk != 128) || (a->dv != 64 && a->dv != 128)) return KDA_ERR_UNSUPPORTED;
+  if (!(a->eps >= 0.f) || !(a->scale >= 0.f)) return KDA_ERR_INVALID_ARGUMENT;
+  if ((int64_t)a->N * a->H > INT32_MAX) return KDA_ERR_UNSUPPORTED;
+  if (a->N > 0) {
+    const void* req[] = {a->q, a->k, a->v, a->g, a->beta, a->state, a->out};
+    for (const void* p : req)
+      if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+    if (a->gate && !aligned16(a->gate)) return KDA_ERR_INVALID_ARGUMENT;
+    if (a->norm_weight && !aligned16(a->norm_weight)) return KDA_ERR_INVALID_ARGUMENT;
+    if (!a->state_indices && a->num_slots < a->N) return KDA_ERR_INVALID_ARGUMENT;
+    if (a->num_slots == 0) return KDA_ERR_INVALID_ARGUMENT;
+  }
+  if (a->N == 0) return KDA_OK;
+  kda_decode_args b = *a;
+  if (!(b.scale > 0.f)) b.scale = 1.0f / sqrtf((float)b.dk);
+  return launch_decode(b, (cudaStream_t)cuda_stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+extern "C" kda_status kda_read_device_error(const void* error_word, void* cuda_stream) {
+  if (!error_word) return KDA_ERR_INVALID_ARGUMENT;
+  if (cudaStreamSynchronize((cudaStream_t)cuda_stream) != cudaSuccess) return KDA_ERR_CUDA;
+  uint32_t w = 0;
+  if (cudaMemcpy(&w, error_word, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return KDA_ERR_CUDA;
+  if (w != 0 && cudaMemset((void*)error_word, 0, sizeof(w)) != cudaSuccess) return KDA_ERR_CUDA;
+  return (kda_status)w;
+}
+
+extern "C" const char* kda_status_string(kda_status s) {
+  switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARGUMENT: return "KDA_ERR_INVALID_ARGUMENT";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+    case KDA_ERR_WORKSPACE_TOO_SMALL: return "KDA_ERR_WORKSPACE_TOO_SMALL";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+    case KDA_ERR_DECAY_OUT_OF_RANGE: return "KDA_ERR_DECAY_OUT_OF_RANGE";
+    case KDA_ERR_BAD_STATE_INDEX: return "KDA_ERR_BAD_STATE_INDEX";
+  }
+  return "KDA_ERR_UNKNOWN";
+}

@@ -1,0 +1,164 @@
+"""The C ABI boundary, without a GPU: libkda.so loads, exports every entry point that
+include/*.h declares, and rejects bad arguments on the host before any CUDA call.
+
+Pointers below are fake (never dereferenced): validation returns before the first
+CUDA call, so these tests run on a machine without a GPU.  cu_seqlens is a real host
+array because the host reads it.
+"""
+import ctypes
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+import linear_attention_serving_rule_b200 as kda
+from linear_attention_serving_rule_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x7F0000000000  # 256-byte aligned, never dereferenced
+
+
+def _declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(kda_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def L():
+    kda.build_library()
+    return kda.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    declared = _declared_functions()
+    assert {"kda_chunk_fwd", "kda_decode_step", "kda_chunk_fwd_workspace_size",
+            "kda_read_device_error", "kda_status_string"} <= declared
+    for name in declared:
+        assert hasattr(L, name), f"libkda.so does not export {name}"
+    assert set(B.EXPORTED) <= declared
+
+
+def test_status_strings(L):
+    for code, name in [(0, "KDA_OK"), (1, "KDA_ERR_INVALID_ARGUMENT"), (3, "KDA_ERR_WORKSPACE_TOO_SMALL"),
+                       (5, "KDA_ERR_TIMEOUT"), (6, "KDA_ERR_DECAY_OUT_OF_RANGE"),
+                       (7, "KDA_ERR_BAD_STATE_INDEX")]:
+        assert kda.kda_status_string(code) == name
+    assert kda.kda_status_string(99) == "KDA_ERR_UNKNOWN"
+
+
+def _args(**kw):
+    a = B.KdaChunkArgs()
+    a.num_seqs, a.total_tokens, a.cu_seqlens = 2, 256, None
+    a.H, a.dk, a.dv, a.dtype = 4, 128, 128, B.KDA_BF16
+    for f in ("q", "k", "v", "g", "beta", "gate", "out"):
+        setattr(a, f, FAKE)
+    a.norm_weight = a.initial_state = a.final_state = None
+    a.scale, a.eps, a.flags, a.split_segments = 0.0, 1e-6, 0, 0
+    a.workspace, a.workspace_bytes = FAKE, 1 << 30
+    for k_, v_ in kw.items():
+        setattr(a, k_, v_)
+    return a
+
+
+def _fwd(L, a):
+    return L.kda_chunk_fwd(ctypes.byref(a), None)
+
+
+def _ws(L, a):
+    n = ctypes.c_size_t(0)
+    rc = L.kda_chunk_fwd_workspace_size(ctypes.byref(a), ctypes.byref(n))
+    return rc, n.value
+
+
+@pytest.mark.parametrize("field", ["q", "k", "v", "g", "beta", "out"])
+def test_null_required_pointer(L, field):
+    assert _fwd(L, _args(**{field: None})) == B.KDA_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.parametrize("field", ["q", "v", "gate", "out"])
+def test_misaligned_pointer(L, field):
+    assert _fwd(L, _args(**{field: FAKE + 2})) == B.KDA_ERR_INVALID_ARGUMENT
+
+
+@pytest.mark.parametrize("dk,dv,code", [(96, 128, B.KDA_ERR_UNSUPPORTED), (128, 32, B.KDA_ERR_UNSUPPORTED),
+                                        (0, 128, B.KDA_ERR_INVALID_ARGUMENT)])
+def test_head_dims(L, dk, dv, code):
+    assert _fwd(L, _args(dk=dk, dv=dv)) == code
+
+
+def test_bad_scalars(L):
+    assert _fwd(L, _args(H=0)) == B.KDA_ERR_INVALID_ARGUMENT
+    assert _fwd(L, _args(dtype=7)) == B.KDA_ERR_INVALID_ARGUMENT
+    assert _fwd(L, _args(eps=-1.0)) == B.KDA_ERR_INVALID_ARGUMENT
+    assert _fwd(L, _args(eps=float("nan"))) == B.KDA_ERR_INVALID_ARGUMENT
+    assert _fwd(L, _args(scale=-0.5)) == B.KDA_ERR_INVALID_ARGUMENT
+    assert _fwd(L, _args(split_segments=-1)) == B.KDA_ERR_INVALID_ARGUMENT
+    assert _fwd(L, _args(total_tokens=255)) == B.KDA_ERR_INVALID_ARGUMENT  # not divisible by num_seqs
+    assert _fwd(L, _args(num_seqs=0, total_tokens=5)) == B.KDA_ERR_INVALID_ARGUMENT
+    assert _fwd(L, _args(total_tokens=1 << 31)) == B.KDA_ERR_UNSUPPORTED
+
+
+def test_cu_seqlens_validation(L):
+    good = np.array([0, 100, 100, 256], dtype=np.int32)
+    bad_start = np.array([1, 100, 100, 256], dtype=np.int32)
+    decreasing = np.array([0, 100, 90, 256], dtype=np.int32)
+    wrong_total = np.array([0, 100, 100, 255], dtype=np.int32)
+    for arr, code in [(bad_start, B.KDA_ERR_INVALID_ARGUMENT), (decreasing, B.KDA_ERR_INVALID_ARGUMENT),
+                      (wrong_total, B.KDA_ERR_INVALID_ARGUMENT)]:
+        assert _fwd(L, _args(num_seqs=3, cu_seqlens=arr.ctypes.data)) == code
+    rc, n = _ws(L, _args(num_seqs=3, cu_seqlens=good.ctypes.data))
+    assert rc == B.KDA_OK and n >= 4
+
+
+def test_workspace_size_and_check(L):
+    rc, n = _ws(L, _args())
+    assert rc == B.KDA_OK and n == 256  # error word only: 8 units fill too little GPU to split 128-token sequences
+    assert _fwd(L, _args(workspace=None)) == B.KDA_ERR_INVALID_ARGUMENT
+    assert _fwd(L, _args(workspace=FAKE + 16)) == B.KDA_ERR_INVALID_ARGUMENT
+    assert _fwd(L, _args(workspace_bytes=n - 1)) == B.KDA_ERR_WORKSPACE_TOO_SMALL
+    # a forced split needs per-segment state buffers
+    rc, n3 = _ws(L, _args(split_segments=3, total_tokens=2 * 1024))
+    assert rc == B.KDA_OK
+    segs = 3 * 2  # 1024 tokens -> 3 segments of 384 (multiple of 64) per sequence
+    assert n3 == 256 + segs * 4 * (128 * 128 + 128 * 256) * 4
+
+
+def test_automatic_split_for_long_context(L):
+    # 1 sequence x 16 heads of 1M tokens: 16 units < half of 148 SMs -> split into 9 segments
+    rc, n = _ws(L, _args(num_seqs=1, total_tokens=1 << 20, H=16))
+    assert rc == B.KDA_OK
+    per_slot = 16 * (128 * 128 + 128 * 256) * 4
+    assert (n - 256) % per_slot == 0 and (n - 256) // per_slot == 9
+
+
+def _dargs(**kw):
+    a = B.KdaDecodeArgs()
+    a.N, a.H, a.dk, a.dv, a.dtype = 8, 4, 128, 128, B.KDA_BF16
+    for f in ("q", "k", "v", "g", "beta", "gate", "state", "out"):
+        setattr(a, f, FAKE)
+    a.norm_weight = a.state_indices = a.error_word = None
+    a.num_slots = 8
+    a.scale, a.eps, a.flags = 0.0, 1e-6, 0
+    for k_, v_ in kw.items():
+        setattr(a, k_, v_)
+    return a
+
+
+def test_decode_validation(L):
+    f = lambda **kw: L.kda_decode_step(ctypes.byref(_dargs(**kw)), None)
+    for field in ("q", "k", "v", "g", "beta", "state", "out"):
+        assert f(**{field: None}) == B.KDA_ERR_INVALID_ARGUMENT
+    assert f(state=FAKE + 4) == B.KDA_ERR_INVALID_ARGUMENT
+    assert f(dk=96) == B.KDA_ERR_UNSUPPORTED
+    assert f(num_slots=7) == B.KDA_ERR_INVALID_ARGUMENT       # identity slots need num_slots >= N
+    assert f(num_slots=0, state_indices=FAKE) == B.KDA_ERR_INVALID_ARGUMENT
+    assert f(N=-1) == B.KDA_ERR_INVALID_ARGUMENT
+    assert f(N=0) == B.KDA_OK                                  # nothing to do, nothing launched
+    assert L.kda_read_device_error(None, None) == B.KDA_ERR_INVALID_ARGUMENT
