@@ -25,7 +25,8 @@
  *
  * Conventions for every entry point:
  *   - Tensor pointers are DEVICE pointers owned by the caller, row-major and
- *     contiguous, 16-byte aligned.  Exceptions are marked HOST.
+ *     contiguous, 16-byte aligned (beta: aligned to its element size).  Exceptions are
+ *     marked HOST.
  *   - The library allocates no memory, never synchronises the stream (except
  *     kda_read_device_error) and launches its kernels on the given cudaStream_t
  *     (passed as void*; NULL = the legacy default stream).
@@ -64,7 +65,7 @@ typedef enum kda_status {
   KDA_ERR_CUDA = 4,               /* a CUDA runtime call or kernel launch failed */
   KDA_ERR_TIMEOUT = 5,            /* (device) a bounded wait inside a kernel ran out */
   KDA_ERR_DECAY_OUT_OF_RANGE = 6, /* (device, checked mode) some g outside [KDA_G_MIN, 0] */
-  KDA_ERR_BAD_STATE_INDEX = 7     /* (device, checked mode) state_indices[n] outside [0, num_slots) */
+  KDA_ERR_BAD_STATE_INDEX = 7     /* (device) state_indices[n] outside [0, num_slots): unit skipped */
 } kda_status;
 
 typedef enum kda_dtype {

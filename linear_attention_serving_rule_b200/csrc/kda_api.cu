@@ -21,6 +21,8 @@ constexpr int kMinAutoSeg = 2048; // automatic split: tokens per segment at leas
 constexpr size_t kErrBytes = 256;
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+// beta is read with scalar loads: element alignment is enough.
+bool aligned_elem(const void* p, kda_dtype dt) { return ((uintptr_t)p & (dt == KDA_BF16 ? 1u : 3u)) == 0; }
 
 struct SeqSpan {
   int32_t tok0, len, seq;
@@ -46,9 +48,10 @@ kda_status validate(const kda_chunk_args* a) {
   if (!(a->eps >= 0.f) || !(a->scale >= 0.f)) return KDA_ERR_INVALID_ARGUMENT;
   if (a->num_seqs == 0 && a->total_tokens != 0) return KDA_ERR_INVALID_ARGUMENT;
   if (a->total_tokens > 0) {
-    const void* req[] = {a->q, a->k, a->v, a->g, a->beta, a->out};
+    const void* req[] = {a->q, a->k, a->v, a->g, a->out};
     for (const void* p : req)
       if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+    if (!a->beta || !aligned_elem(a->beta, a->dtype)) return KDA_ERR_INVALID_ARGUMENT;
     if (a->gate && !aligned16(a->gate)) return KDA_ERR_INVALID_ARGUMENT;
   }
   if (a->norm_weight && !aligned16(a->norm_weight)) return KDA_ERR_INVALID_ARGUMENT;
@@ -170,6 +173,7 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
   float* ws = (float*)((char*)a->workspace + kErrBytes);
   p.ws_state = L.slots ? ws : nullptr;
   p.ws_local = L.slots ? ws + (size_t)L.slots * a->H * a->dk * a->dv : nullptr;
+  p.total_tokens = a->total_tokens;
   p.H = a->H; p.dk = a->dk; p.dv = a->dv;
   p.scale = a->scale > 0.f ? a->scale : 1.0f / sqrtf((float)a->dk);
   p.eps = a->eps;
@@ -178,7 +182,9 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
   if (cudaMemsetAsync(a->workspace, 0, sizeof(uint32_t), stream) != cudaSuccess) return KDA_ERR_CUDA;
   if (a->num_seqs == 0) return KDA_OK;
 
-  const bool use_tc = false;
+  // bf16 with dk = dv = 128 runs on the tensor cores; everything else (and the split's
+  // augmented pass 1) on the fp32 CUDA-core kernel.
+  const bool use_tc = a->dtype == KDA_BF16 && a->dk == 128 && a->dv == 128 && !(a->flags & KDA_FLAG_FORCE_SIMT);
 
   // Pass 1 of split sequences: the head segment from the true initial state, and the
   // other non-final segments from [0 | I] (local state and transition matrix).
@@ -201,7 +207,7 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
     }
   }
   cudaError_t e = cudaSuccess;
-  if (!head.empty()) e = run_segments(head, p, a->dtype, false, stream);
+  if (!head.empty()) e = run_segments(head, p, a->dtype, use_tc, stream);
   if (e == cudaSuccess && !local.empty()) e = run_segments(local, p, a->dtype, false, stream);
   if (e == cudaSuccess && L.any_split) {
     // combine: S_start(q+1) = M_q S_start(q) + S_loc(q), sequential over q per (sequence, head)
@@ -231,9 +237,10 @@ extern "C" kda_status kda_decode_step(const kda_decode_args* a, void* cuda_strea
   if (!(a->eps >= 0.f) || !(a->scale >= 0.f)) return KDA_ERR_INVALID_ARGUMENT;
   if ((int64_t)a->N * a->H > INT32_MAX) return KDA_ERR_UNSUPPORTED;
   if (a->N > 0) {
-    const void* req[] = {a->q, a->k, a->v, a->g, a->beta, a->state, a->out};
+    const void* req[] = {a->q, a->k, a->v, a->g, a->state, a->out};
     for (const void* p : req)
       if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+    if (!a->beta || !aligned_elem(a->beta, a->dtype)) return KDA_ERR_INVALID_ARGUMENT;
     if (a->gate && !aligned16(a->gate)) return KDA_ERR_INVALID_ARGUMENT;
     if (a->norm_weight && !aligned16(a->norm_weight)) return KDA_ERR_INVALID_ARGUMENT;
     if (!a->state_indices && a->num_slots < a->N) return KDA_ERR_INVALID_ARGUMENT;

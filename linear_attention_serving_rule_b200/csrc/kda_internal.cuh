@@ -56,6 +56,7 @@ struct ChunkParams {
   float* ws_state;     // split: per-slot [dk, dv] start states (pass 2 reads), or null
   float* ws_local;     // split: per-slot [dk, dv + dk] (S_loc | M) from pass 1, or null
   uint32_t* error_word;
+  int64_t total_tokens;  // rows of the packed tensors (tensor-map extent)
   int32_t H, dk, dv;
   float scale, eps;
   uint32_t flags;

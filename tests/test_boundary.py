@@ -87,6 +87,12 @@ def test_misaligned_pointer(L, field):
     assert _fwd(L, _args(**{field: FAKE + 2})) == B.KDA_ERR_INVALID_ARGUMENT
 
 
+def test_beta_needs_element_alignment_only(L):
+    assert _ws(L, _args(beta=FAKE + 2))[0] == B.KDA_OK
+    assert _fwd(L, _args(beta=FAKE + 1)) == B.KDA_ERR_INVALID_ARGUMENT
+    assert _fwd(L, _args(beta=FAKE + 2, dtype=B.KDA_F32)) == B.KDA_ERR_INVALID_ARGUMENT
+
+
 @pytest.mark.parametrize("dk,dv,code", [(96, 128, B.KDA_ERR_UNSUPPORTED), (128, 32, B.KDA_ERR_UNSUPPORTED),
                                         (0, 128, B.KDA_ERR_INVALID_ARGUMENT)])
 def test_head_dims(L, dk, dv, code):

@@ -195,3 +195,19 @@ def test_long_context_prefix_and_full_run():
         assert rel_l2(fin[u].cpu().numpy(), ref[u][1]) <= TOL_STATE_BF16, u
         o, _ = gpu_unit(out, None, full.cu_seqlens, *u)
         assert rel_l2(o[-4096:], ref[u][0][-4096:]) <= TOL_OUT_BF16, u
+
+
+def test_forced_timeout_reports_and_recovers():
+    """The test-only flag makes the tensor-core kernel's bounded waits give up at once: the call
+    reports KDA_ERR_TIMEOUT in the error word, drains its own copies, frees TMEM and returns;
+    the next call on the same context is correct."""
+    inp = synth.make_prefill(H=2, dk=128, dv=128, dtype="bf16", seed=37, device="cuda",
+                             lengths=np.array([300, 100]), gate=True, init_state=True)
+    _, _, ws = kda.kda_chunk_fwd(inp.q, inp.k, inp.v, inp.g, inp.beta, gate=inp.gate,
+                                 cu_seqlens=inp.cu_seqlens, initial_state=inp.initial_state,
+                                 flags=kda.KDA_FLAG_TEST_FORCE_TIMEOUT)
+    assert kda.kda_read_device_error(ws) == kda.binding.KDA_ERR_TIMEOUT
+    out, fin = _run(inp)
+    o_ref, f_ref = oracle_full(inp)
+    assert rel_l2(host(out), o_ref) <= TOL_OUT_BF16
+    assert rel_l2(host(fin), f_ref) <= TOL_STATE_BF16
