@@ -21,12 +21,16 @@
 // operand Kc_a = k e^{r_a - gamma} over the first 16(a+1) tokens; one M=128 UMMA per a
 // produces A (rows 0-63) and P (rows 64-127) from the stacked operand [k; q] e^{gamma - r_own}.
 //
-// Work split (160 threads): warp 4 is the TMA producer (q, k, g | v | gate tiles, released per
-// group as soon as the chunk no longer needs them); warps 0-3 are the compute warpgroup:
-// thread i owns TMEM lane i and row i of the fp32 state S (kept in registers), builds the
-// decayed bf16 operands, the UT inverse T', and runs the epilogue; thread 0 issues the UMMAs.
+// Work split (288 threads): warp 8 is the TMA producer (k and q land interleaved as one
+// 128-row tile, g and v beside them; q/k/g are handed back as soon as the Gram UMMAs have
+// read them, v after the W/U' UMMAs); warps 0-7 are two compute warpgroups.  Warp w owns
+// TMEM lane quarter w % 4 and works on column half w / 4, so every CUDA-core phase (decay
+// prep, Gram read-out, UT inverse, -W/U conversion, state copy, epilogue) runs on 256
+// threads; thread 0 issues the UMMAs.  The gate logits are read straight from global memory
+// by the epilogue.
 //
-// TMEM (512 columns allocated): [0,128) K^T U (M=128); [128,288) A|P (M=128, N = 16,32,48,64);
+// TMEM (512 columns allocated): [0,128) the fp32 state S (M=128; decayed in place while the
+// Gram UMMAs run, then K^T U accumulated onto it); [128,288) A|P (M=128, N = 16,32,48,64);
 // [288,416) W / O at lane offset 0 and U' -> U at lane offset 16 (two interleaved M=64 tiles).
 //
 // Every wait is bounded (%globaltimer): on expiry the kernel records KDA_ERR_TIMEOUT, stops
@@ -45,44 +49,47 @@ using namespace ptx;
 constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int DV = 128;
-constexpr int kCompute = 128;
-constexpr int kThreads = 160;
+constexpr int kCompute = 256;
+constexpr int kThreads = 288;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_Q = 0, OFF_K = 16384, OFF_G = 32768, OFF_V = 49152, OFF_GATE = 65536;
-constexpr uint32_t OFF_S = 81920;    // bf16 state, MN-major [dk rows][dv], two 16 KB column blocks
-constexpr uint32_t OFF_R = 114688;   // 72 KB region reused across the phases of a chunk
-// phase A (decayed Gram operands)
-constexpr uint32_t R_KQ = 0;                                        // [k; q] e^{gamma - r_own}, 128 rows
-// Kc_a (16(a+1) rows) at 32768, 36864, 45056, 57344
-__host__ __device__ constexpr uint32_t r_kc(int a) { return a == 0 ? 32768u : a == 1 ? 36864u : a == 2 ? 45056u : 57344u; }
-// phase B (inverse) and later
-constexpr uint32_t R_AF = 0, R_TF = 16640;                          // fp32 [64][65]
-constexpr uint32_t R_KT = 0, R_QT = 16384, R_KH = 32768;            // e^g k, e^g q, e^{gC-g} k
-constexpr uint32_t R_W = 0, R_U = 0;                                // -W, then U (bf16)
-constexpr uint32_t R_TP = 49152, R_P = 57344, R_Y = 65536;          // T', P (bf16), scratch
-constexpr uint32_t OFF_MISC = OFF_R + 73728;                        // 188416
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 4096 + 1024;             // + misc + alignment slack
-constexpr int LDF = 65;                                             // fp32 row stride of A, T
+constexpr uint32_t OFF_KQ = 0;       // k rows 0-63 | q rows 64-127 (TMA), then [k; q] e^{gamma - r_own} in place
+constexpr uint32_t OFF_G = 32768;    // g (TMA)
+constexpr uint32_t OFF_V = 49152;    // v (TMA), B operand of U' = T' V
+constexpr uint32_t OFF_KC = 65536;   // Kc_0..Kc_3 (40 KB); then fp32 A and T of the inverse
+constexpr uint32_t OFF_KT = 106496;  // e^{gamma} k; then -W; then U
+constexpr uint32_t OFF_QT = 122880;  // e^{gamma} q
+constexpr uint32_t OFF_KH = 139264;  // e^{gamma_C - gamma} k
+constexpr uint32_t OFF_S = 155648;   // bf16 state, MN-major [dk rows][dv], two 16 KB column blocks
+constexpr uint32_t OFF_TP = 188416;  // T' = T Diag(beta), bf16 [64][64]
+constexpr uint32_t OFF_P = 196608;   // P (causally masked), bf16 [64][64]
+constexpr uint32_t OFF_MISC = 204800;
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 8192 + 1024;
+constexpr uint32_t OFF_TF = OFF_KC + 16640;  // fp32 T, after fp32 A (both [64][65])
+constexpr int LDF = 65;
 
-constexpr uint32_t TM_KU = 0, TM_AP = 128, TM_WU = 288;
+constexpr uint32_t TM_S = 0, TM_AP = 128, TM_WU = 288;
+
+// Kc_a (16(a+1) rows, two column blocks of 16(a+1) x 128 bytes) inside OFF_KC
+__host__ __device__ constexpr uint32_t kc_off(int a) { return a == 0 ? 0u : a == 1 ? 4096u : a == 2 ? 12288u : 24576u; }
 // column offset of the A|P accumulator of sub-tile a (N = 16, 32, 48, 64)
 __host__ __device__ constexpr uint32_t ap_off(int a) { return a == 0 ? 0u : a == 1 ? 16u : a == 2 ? 48u : 96u; }
 
 struct Misc {
-  uint64_t full_qkg, full_v, full_gate, empty_qkg, empty_v, empty_gate, mma;
+  uint64_t full_qkg, full_v, empty_qkg, empty_v, mma;
   uint32_t tmem_base;
   int32_t abort;
   float beta[C];
-  float2 tot[64];
-  float ref[5][DK];   // r_0..r_3 and gamma_C per channel (log2 units)
-  float ec[DK];       // e^{gamma_C}
+  float se[4][DK];  // e^{decay over sub-tile m}, per channel
+  float ec[DK];     // e^{gamma_C}
+  float ss[2][C];   // epilogue: partial sums of squares of the two column halves
+  float y[768];     // inverse scratch
 };
-static_assert(sizeof(Misc) <= 4096, "misc block too large");
+static_assert(sizeof(Misc) <= 8192, "misc block too large");
 
 struct TcMaps {
-  CUtensorMap q, k, g, v, gate;
+  CUtensorMap q, k, g, v;
 };
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -115,20 +122,22 @@ __device__ __forceinline__ uint32_t f2_to_bf2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+__device__ __forceinline__ void unpack8(uint4 u, float (&f)[8]) {
+  float2 a = bf2_to_f2(u.x), b = bf2_to_f2(u.y), c = bf2_to_f2(u.z), d = bf2_to_f2(u.w);
+  f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y; f[4] = c.x; f[5] = c.y; f[6] = d.x; f[7] = d.y;
+}
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  return make_uint4(f2_to_bf2(f[0], f[1]), f2_to_bf2(f[2], f[3]), f2_to_bf2(f[4], f[5]), f2_to_bf2(f[6], f[7]));
+}
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-__device__ __forceinline__ void st_u32(uint8_t* base, uint32_t off, uint32_t v) {
-  *reinterpret_cast<uint32_t*>(base + off) = v;
-}
-__device__ __forceinline__ uint32_t ld_u32(const uint8_t* base, uint32_t off) {
-  return *reinterpret_cast<const uint32_t*>(base + off);
-}
+__device__ __forceinline__ uint4& at16(uint8_t* base, uint32_t off) { return *reinterpret_cast<uint4*>(base + off); }
 
-// Issue the K loop of one UMMA: A and B descriptors advance by (a_step, b_step) bytes per
-// 16-wide K step; K-major 128-wide operands jump to their second 64-column block after 4 steps.
+// Issue the K loop of one UMMA.  K-major operands step 32 bytes per 16-wide K step and jump to
+// their second 64-column block (blk bytes away) after 4 steps; MN-major ones step 2048 bytes.
 __device__ __forceinline__ void umma_k_loop(uint32_t d, uint32_t a_addr, uint32_t a_lbo, bool a_kmajor,
                                             uint32_t a_blk, uint32_t b_addr, uint32_t b_lbo, bool b_kmajor,
                                             uint32_t b_blk, int ksteps, uint32_t idesc, bool accumulate) {
@@ -145,7 +154,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Misc* m = reinterpret_cast<Misc*>(sm + OFF_MISC);
-  uint8_t* R = sm + OFF_R;
   const uint32_t sm_u = smem_u32(sm);
 
   const int tid = threadIdx.x;
@@ -160,8 +168,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nchunks = (seg.len + C - 1) / C;
 
   if (tid == 0) {
-    mbar_init(&m->full_qkg, 1); mbar_init(&m->full_v, 1); mbar_init(&m->full_gate, 1);
-    mbar_init(&m->empty_qkg, 1); mbar_init(&m->empty_v, 1); mbar_init(&m->empty_gate, 1);
+    mbar_init(&m->full_qkg, 1); mbar_init(&m->full_v, 1);
+    mbar_init(&m->empty_qkg, 1); mbar_init(&m->empty_v, 1);
     mbar_init(&m->mma, 1);
     m->abort = 0;
     fence_mbar_init();
@@ -170,27 +178,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(&m->tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.g); prefetch_tmap(&maps.v);
-    if (has_gate) prefetch_tmap(&maps.gate);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = m->tmem_base;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ===================================================================== TMA producer
     if (lane == 0) {
-      int iq = -1, iv = -1, ig = -1;  // last chunk whose q/k/g, v, gate loads were issued
+      int iq = -1, iv = -1;  // last chunk whose q/k/g and v loads were issued
       for (int j = 0; j < nchunks; ++j) {
         const int32_t tok = seg.tok0 + j * C;
         const uint32_t par = (uint32_t)((j & 1) ^ 1);
         if (!wait_bounded(&m->empty_qkg, par, m, drain_limit, p.error_word)) break;
         mbar_arrive_expect_tx(&m->full_qkg, 3 * 16384);
         for (int hf = 0; hf < 2; ++hf) {
-          tma_load_3d(sm + OFF_Q + hf * 8192, &maps.q, &m->full_qkg, hf * 64, h, tok);
-          tma_load_3d(sm + OFF_K + hf * 8192, &maps.k, &m->full_qkg, hf * 64, h, tok);
+          tma_load_3d(sm + OFF_KQ + hf * 16384, &maps.k, &m->full_qkg, hf * 64, h, tok);
+          tma_load_3d(sm + OFF_KQ + hf * 16384 + 8192, &maps.q, &m->full_qkg, hf * 64, h, tok);
           tma_load_3d(sm + OFF_G + hf * 8192, &maps.g, &m->full_qkg, hf * 64, h, tok);
         }
         iq = j;
@@ -198,48 +205,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&m->full_v, 16384);
         for (int hf = 0; hf < 2; ++hf) tma_load_3d(sm + OFF_V + hf * 8192, &maps.v, &m->full_v, hf * 64, h, tok);
         iv = j;
-        if (has_gate) {
-          if (!wait_bounded(&m->empty_gate, par, m, drain_limit, p.error_word)) break;
-          mbar_arrive_expect_tx(&m->full_gate, 16384);
-          for (int hf = 0; hf < 2; ++hf)
-            tma_load_3d(sm + OFF_GATE + hf * 8192, &maps.gate, &m->full_gate, hf * 64, h, tok);
-          ig = j;
-        }
       }
       // drain: after an abort, wait (bounded, regardless of the abort) for the loads issued
       if (*(volatile int32_t*)&m->abort) {
         if (iq >= 0) wait_bounded(&m->full_qkg, (uint32_t)(iq & 1), m, drain_limit, p.error_word, false);
         if (iv >= 0) wait_bounded(&m->full_v, (uint32_t)(iv & 1), m, drain_limit, p.error_word, false);
-        if (ig >= 0) wait_bounded(&m->full_gate, (uint32_t)(ig & 1), m, drain_limit, p.error_word, false);
       }
     }
   } else {
-    // ===================================================================== compute warpgroup
-    float S[DV];  // row `tid` of the fp32 state
+    // ===================================================================== compute warpgroups
+    const int q4 = warp & 3;   // TMEM lane quarter
+    const int wg = warp >> 2;  // column half
+    const int row = 32 * q4 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
     const size_t unit_state = (size_t)DK * DV;
-    {
-      const float* src = nullptr;
-      if (seg.role == kRoleWhole || seg.role == kRoleHead) {
-        if (p.initial_state) src = p.initial_state + ((size_t)seg.seq * H + h) * unit_state;
-      } else if (seg.role == kRoleFromWs) {
-        src = p.ws_state + ((size_t)seg.slot * H + h) * unit_state;
-      }
-#pragma unroll
-      for (int c = 0; c < DV; c += 4) {
-        float4 x = src ? *reinterpret_cast<const float4*>(src + (size_t)tid * DV + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-        S[c] = x.x; S[c + 1] = x.y; S[c + 2] = x.z; S[c + 3] = x.w;
-      }
-#pragma unroll
-      for (int c = 0; c < DV; c += 2) st_u32(sm, OFF_S + sw128_off(tid, c, 16384), f2_to_bf2(S[c], S[c + 1]));
-    }
     const bool write_out = (seg.role == kRoleWhole || seg.role == kRoleFromWs);
-    const int pr = tid & 63, hh = tid >> 6;  // channel pair (2pr, 2pr+1) and token half for the scans
-    const int c0 = 2 * pr;
-    uint32_t mph = 0;  // UMMA barrier phase
+    uint32_t mph = 0;
     bool ok = true;
 
     auto sync_wg = [&]() { named_bar_sync(1, kCompute); };
-    // thread 0 waits, then the warpgroup learns the outcome (uniform abort decision)
+    // thread 0 waits, then both warpgroups learn the outcome (uniform abort decision)
     auto wg_wait = [&](uint64_t* bar, uint32_t par) -> bool {
       if (tid == 0) wait_bounded(bar, par, m, limit, p.error_word);
       sync_wg();
@@ -252,6 +237,42 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       return r;
     };
+    auto sync_for_mma = [&]() {
+      fence_proxy_async_smem();
+      tc_fence_before();
+      sync_wg();
+    };
+
+    // ---------------------------------------------------------------- start state -> TMEM + bf16 copy
+    {
+      const float* src = nullptr;
+      if (seg.role == kRoleWhole || seg.role == kRoleHead) {
+        if (p.initial_state) src = p.initial_state + ((size_t)seg.seq * H + h) * unit_state;
+      } else if (seg.role == kRoleFromWs) {
+        src = p.ws_state + ((size_t)seg.slot * H + h) * unit_state;
+      }
+#pragma unroll
+      for (int hb = 0; hb < 2; ++hb) {
+        const int c0 = wg * 64 + hb * 32;
+        uint32_t v[32];
+#pragma unroll
+        for (int jj = 0; jj < 32; jj += 4) {
+          float4 x = src ? *reinterpret_cast<const float4*>(src + (size_t)row * DV + c0 + jj)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[jj] = __float_as_uint(x.x); v[jj + 1] = __float_as_uint(x.y);
+          v[jj + 2] = __float_as_uint(x.z); v[jj + 3] = __float_as_uint(x.w);
+        }
+        tmem_st32(tl + TM_S + c0, v);
+#pragma unroll
+        for (int oc = 0; oc < 4; ++oc) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
+          at16(sm, OFF_S + sw128_oct(row, (c0 >> 3) + oc, 16384)) = pack8(f);
+        }
+      }
+      tmem_wait_st();
+    }
 
     for (int j = 0; j < nchunks && ok; ++j) {
       const int L = min(C, seg.len - j * C);
@@ -264,129 +285,191 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!wg_wait(&m->full_qkg, par)) { ok = false; break; }
 
-      // ---------------------------------------------------------------- prep 1: Gram operands
-      float gam[32][2];
+      // ---------------------------------------------------------------- decay prep (one pass)
+      // thread: channels 8o .. 8o+7, tokens t0 .. t0+3 of sub-tile b
       {
-        float a0 = 0.f, a1 = 0.f;
+        const int qq = tid & 3, o = (tid >> 2) & 15, b = tid >> 6;
+        const int t0 = 16 * b + 4 * qq;
+        float gl[4][8];  // inclusive cumulative log2-decay from the sub-tile start
+        float acc[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int t = 32 * hh + i;
-          float2 gv = make_float2(0.f, 0.f);
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int t = t0 + i;
+          float g8[8];
           if (t < L) {
-            gv = bf2_to_f2(ld_u32(sm, OFF_G + sw128_off(t, c0, 8192)));
-            if (checked && !(gv.x >= KDA_G_MIN && gv.x <= 0.f && gv.y >= KDA_G_MIN && gv.y <= 0.f))
-              report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
+            unpack8(at16(sm, OFF_G + sw128_oct(t, o, 8192)), g8);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) g8[e] = 0.f;
           }
-          a0 += gv.x * kLog2e; a1 += gv.y * kLog2e;
-          gam[i][0] = a0; gam[i][1] = a1;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (checked && !(g8[e] >= KDA_G_MIN && g8[e] <= 0.f)) report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
+            acc[e] += g8[e] * kLog2e;
+            gl[i][e] = acc[e];
+          }
         }
-        if (hh == 0) m->tot[pr] = make_float2(a0, a1);
-      }
-      sync_wg();
-      if (hh == 1) {
-        const float2 o = m->tot[pr];
+        // prefix over the four threads of the sub-tile (lanes differing in bits 0-1)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) { gam[i][0] += o.x; gam[i][1] += o.y; }
-        m->ref[3][c0] = gam[15][0]; m->ref[3][c0 + 1] = gam[15][1];
-        m->ref[4][c0] = gam[31][0]; m->ref[4][c0 + 1] = gam[31][1];
-      } else {
-        m->ref[0][c0] = 0.f; m->ref[0][c0 + 1] = 0.f;
-        m->ref[1][c0] = gam[15][0]; m->ref[1][c0 + 1] = gam[15][1];
-        m->ref[2][c0] = gam[31][0]; m->ref[2][c0 + 1] = gam[31][1];
-      }
-      sync_wg();
-      {
-        float r[4][2];
+        for (int e = 0; e < 8; ++e) {
+          float x = acc[e];
+          float y = __shfl_up_sync(0xffffffffu, x, 1, 4);
+          if (qq >= 1) x += y;
+          y = __shfl_up_sync(0xffffffffu, x, 2, 4);
+          if (qq >= 2) x += y;
+          const float excl = x - acc[e];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) { r[a][0] = m->ref[a][c0]; r[a][1] = m->ref[a][c0 + 1]; }
+          for (int i = 0; i < 4; ++i) gl[i][e] += excl;
+          if (qq == 3) m->se[b][8 * o + e] = ex2(x);  // decay over the whole sub-tile
+        }
+        sync_wg();
+        // Per-channel factors, split so that no product of an O(1) value with an underflowed
+        // factor is lost: with se_m = e^{decay over sub-tile m},
+        //   Eb   = e^{r_b}                       = prod_{m<b} se_m
+        //   Rh_a = e^{r_a - r_{b+1}}  (a > b)    = prod_{b<m<a} se_m
+        //   Ehi  = e^{gamma_C - r_{b+1}}         = prod_{m>b} se_m
+        // and per token ix * se_b = e^{r_{b+1} - gamma_t} lies in [e^-80, 1].
+        float Eb[8], Ehi[8], sb[8], Rh[4][8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int t = 32 * hh + i;
-          const int b = t >> 4;  // = 2 hh + (i >> 4)
-          float2 kv = make_float2(0.f, 0.f), qv = kv;
-          if (t < L) {
-            kv = bf2_to_f2(ld_u32(sm, OFF_K + sw128_off(t, c0, 8192)));
-            qv = bf2_to_f2(ld_u32(sm, OFF_Q + sw128_off(t, c0, 8192)));
+        for (int e = 0; e < 8; ++e) {
+          float se[4];
+#pragma unroll
+          for (int mm = 0; mm < 4; ++mm) se[mm] = m->se[mm][8 * o + e];
+          float eb = 1.f, ehi = 1.f, r = 1.f;
+#pragma unroll
+          for (int mm = 0; mm < 4; ++mm) {
+            if (mm < b) eb *= se[mm];
+            if (mm > b) ehi *= se[mm];
+            Rh[mm][e] = r;  // for mm > b: prod over b < m < mm
+            if (mm > b) r *= se[mm];
           }
-          const float x0 = ex2(gam[i][0] - r[b][0]), x1 = ex2(gam[i][1] - r[b][1]);
-          const float ix0 = ex2(r[b][0] - gam[i][0]), ix1 = ex2(r[b][1] - gam[i][1]);
-          st_u32(R, R_KQ + sw128_off(t, c0, 16384), f2_to_bf2(kv.x * x0, kv.y * x1));
-          st_u32(R, R_KQ + sw128_off(64 + t, c0, 16384), f2_to_bf2(qv.x * x0, qv.y * x1));
+          Eb[e] = eb; Ehi[e] = ehi;
+          sb[e] = b == 0 ? se[0] : b == 1 ? se[1] : b == 2 ? se[2] : se[3];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int t = t0 + i;
+          float kf[8], qf[8];
+          if (t < L) {
+            unpack8(at16(sm, OFF_KQ + sw128_oct(t, o, 16384)), kf);
+            unpack8(at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)), qf);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) { kf[e] = 0.f; qf[e] = 0.f; }
+          }
+          float x[8], ix[8], ixs[8], f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) { x[e] = ex2(gl[i][e]); ix[e] = ex2(-gl[i][e]); ixs[e] = ix[e] * sb[e]; }
+          const uint32_t o64 = sw128_oct(t, o, 8192);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = kf[e] * x[e];
+          at16(sm, OFF_KQ + sw128_oct(t, o, 16384)) = pack8(f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = qf[e] * x[e];
+          at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)) = pack8(f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = kf[e] * x[e] * Eb[e];
+          at16(sm, OFF_KT + o64) = pack8(f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = qf[e] * x[e] * Eb[e];
+          at16(sm, OFF_QT + o64) = pack8(f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = kf[e] * ixs[e] * Ehi[e];
+          at16(sm, OFF_KH + o64) = pack8(f);
 #pragma unroll
           for (int a = 0; a < 4; ++a) {
             if (a >= b) {
-              const float f0 = ix0 * ex2(r[a][0] - r[b][0]), f1 = ix1 * ex2(r[a][1] - r[b][1]);
-              st_u32(R, r_kc(a) + sw128_off(t, c0, 16 * (a + 1) * 128), f2_to_bf2(kv.x * f0, kv.y * f1));
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = (a == b) ? kf[e] * ix[e] : kf[e] * ixs[e] * Rh[a][e];
+              at16(sm, OFF_KC + kc_off(a) + sw128_oct(t, o, 2048u * (a + 1))) = pack8(f);
             }
           }
         }
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      sync_wg();
+      if (tid < DK) m->ec[tid] = m->se[0][tid] * m->se[1][tid] * m->se[2][tid] * m->se[3][tid];
+      sync_for_mma();
       // ---------------------------------------------------------------- UMMA: A | P
       if (tid == 0) {
         tc_fence_after();
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
           const uint32_t n = 16u * (a + 1);
-          umma_k_loop(tmem + TM_AP + ap_off(a), sm_u + OFF_R + R_KQ, 16, true, 16384, sm_u + OFF_R + r_kc(a), 16,
-                      true, n * 128u, 8, idesc_bf16_f32(128, n, 0, 0), false);
+          umma_k_loop(tmem + TM_AP + ap_off(a), sm_u + OFF_KQ, 16, true, 16384, sm_u + OFF_KC + kc_off(a), 16, true,
+                      n * 128u, 8, idesc_bf16_f32(128, n, 0, 0), false);
         }
+        umma_commit(&m->mma);
       }
-      if (!mma_commit_wait()) { ok = false; break; }
+      // while the Gram UMMAs run: decay the fp32 state in place, S <- Diag(e^{gamma_C}) S
+      {
+        const float ec = m->ec[row];
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+          const uint32_t col = TM_S + wg * 64 + hb * 32;
+          uint32_t v[32];
+          tmem_ld32(tl + col, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) v[jj] = __float_as_uint(__uint_as_float(v[jj]) * ec);
+          tmem_st32(tl + col, v);
+        }
+        tmem_wait_st();
+      }
+      {
+        const bool r = wg_wait(&m->mma, mph & 1u);
+        ++mph;
+        tc_fence_after();
+        if (!r) { ok = false; break; }
+      }
+      if (tid == 0) mbar_arrive(&m->empty_qkg);  // k, q, g fully consumed
 
       // ---------------------------------------------------------------- read A (beta-scaled) and P
       {
-        float* Af = reinterpret_cast<float*>(R + R_AF);
-        const int wq = warp & 1;            // subtiles 2wq, 2wq+1 of this warp's 32 rows
-        const bool isP = warp >= 2;
-        const int t = (warp & 1) * 32 + lane;  // row within A or P
+        float* Af = reinterpret_cast<float*>(sm + OFF_KC);
+        const bool isP = q4 >= 2;
+        const int t = (q4 & 1) * 32 + lane;
+        const int a = 2 * (q4 & 1) + wg;  // the sub-tile whose columns this warp loads
+        const bool mine = (t >> 4) == a;
         const float bt = m->beta[t];
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
 #pragma unroll
-        for (int as = 0; as < 2; ++as) {
-          const int a = 2 * wq + as;
+        for (int kb = 0; kb < 4; ++kb) {
+          if (kb <= a) {
+            uint32_t v[16];
+            tmem_ld16(tl + TM_AP + ap_off(a) + 16 * kb, v);
+            tmem_wait_ld();
+            if (mine) {
+              if (!isP) {
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            if (kb <= a) {
-              uint32_t v[16];
-              tmem_ld16(lane_base + TM_AP + ap_off(a) + 16 * kb, v);
-              tmem_wait_ld();
-              if ((t >> 4) == a) {
-                if (!isP) {
+                for (int jj = 0; jj < 16; ++jj) {
+                  const int s = 16 * kb + jj;
+                  Af[t * LDF + s] = (s < t) ? bt * __uint_as_float(v[jj]) : 0.f;
+                }
+              } else {
 #pragma unroll
-                  for (int jj = 0; jj < 16; ++jj) {
-                    const int s = 16 * kb + jj;
-                    Af[t * LDF + s] = (s < t) ? bt * __uint_as_float(v[jj]) : 0.f;
-                  }
-                } else {
+                for (int oc = 0; oc < 2; ++oc) {
+                  float f[8];
 #pragma unroll
-                  for (int jj = 0; jj < 16; jj += 2) {
-                    const int s = 16 * kb + jj;
-                    const float p0 = (s <= t) ? __uint_as_float(v[jj]) : 0.f;
-                    const float p1 = (s + 1 <= t) ? __uint_as_float(v[jj + 1]) : 0.f;
-                    st_u32(R, R_P + sw128_off(t, s, 8192), f2_to_bf2(p0, p1));
-                  }
+                  for (int e = 0; e < 8; ++e) f[e] = (16 * kb + 8 * oc + e <= t) ? __uint_as_float(v[8 * oc + e]) : 0.f;
+                  at16(sm, OFF_P + sw128_oct(t, 2 * kb + oc, 8192)) = pack8(f);
                 }
               }
             }
           }
         }
-        if (isP) {  // columns past the row's sub-tile are zero
+        if (isP && mine) {
 #pragma unroll
-          for (int s = 0; s < C; s += 2)
-            if (s >= 16 * ((t >> 4) + 1)) st_u32(R, R_P + sw128_off(t, s, 8192), 0u);
+          for (int oc = 0; oc < 8; ++oc)
+            if (oc >= 2 * (a + 1)) at16(sm, OFF_P + sw128_oct(t, oc, 8192)) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      tc_fence_before();
       sync_wg();
 
-      // ---------------------------------------------------------------- UT inverse
+      // ---------------------------------------------------------------- UT inverse: T' = (I + Diag(beta) A)^-1 Diag(beta)
       {
-        const float* Lf = reinterpret_cast<const float*>(R + R_AF);
-        float* Tf = reinterpret_cast<float*>(R + R_TF);
-        float* Y = reinterpret_cast<float*>(R + R_Y);
+        const float* Lf = reinterpret_cast<const float*>(sm + OFF_KC);
+        float* Tf = reinterpret_cast<float*>(sm + OFF_TF);
+        float* Y = m->y;
         if (tid < 64) {  // diagonal 16x16 blocks by forward substitution, one column per thread
           const int a = tid >> 4, jc = tid & 15, o = 16 * a;
           float col[16];
@@ -397,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (i > jc) {
               float acc = 0.f;
 #pragma unroll
-              for (int mm = 0; mm < 16; ++mm)
+              for (int mm = 0; mm < 15; ++mm)
                 if (mm < i && mm >= jc) acc += Lf[(o + i) * LDF + o + mm] * col[mm];
               col[i] = -acc;
             }
@@ -406,62 +489,39 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 16; ++i) Tf[(o + i) * LDF + o + jc] = col[i];
         }
         sync_wg();
-        for (int d = 1; d <= 3; ++d) {  // off-diagonal blocks at distance d
+        for (int d = 1; d <= 3; ++d) {  // off-diagonal blocks at block distance d
           const int nel = (4 - d) * 256;
           for (int e = tid; e < nel; e += kCompute) {
             const int b = e >> 8, i = (e >> 4) & 15, jc = e & 15, a = b + d;
+            const float* lrow = Lf + (16 * a + i) * LDF;
             float acc = 0.f;
-            for (int cc = 16 * b; cc < 16 * a; ++cc) acc += Lf[(16 * a + i) * LDF + cc] * Tf[cc * LDF + 16 * b + jc];
+            for (int cc = 16 * b; cc < 16 * a; ++cc) acc += lrow[cc] * Tf[cc * LDF + 16 * b + jc];
             Y[e] = acc;
           }
           sync_wg();
           for (int e = tid; e < nel; e += kCompute) {
             const int b = e >> 8, i = (e >> 4) & 15, jc = e & 15, a = b + d;
+            const float* trow = Tf + (16 * a + i) * LDF + 16 * a;
             float acc = 0.f;
-            for (int kk = 0; kk <= i; ++kk) acc += Tf[(16 * a + i) * LDF + 16 * a + kk] * Y[(b << 8) + (kk << 4) + jc];
+            for (int kk = 0; kk <= i; ++kk) acc += trow[kk] * Y[(b << 8) + (kk << 4) + jc];
             Tf[(16 * a + i) * LDF + 16 * b + jc] = -acc;
           }
           sync_wg();
         }
-        // T' = T Diag(beta), bf16, K-major [64 rows][64]
-        for (int e = tid; e < C * C / 2; e += kCompute) {
-          const int i = e >> 5, jc = (e & 31) * 2;
-          const float t0 = (jc <= i) ? Tf[i * LDF + jc] * m->beta[jc] : 0.f;
-          const float t1 = (jc + 1 <= i) ? Tf[i * LDF + jc + 1] * m->beta[jc + 1] : 0.f;
-          st_u32(R, R_TP + sw128_off(i, jc, 8192), f2_to_bf2(t0, t1));
-        }
-      }
-      sync_wg();
-
-      // ---------------------------------------------------------------- prep 2: e^g k, e^g q, e^{gC-g} k
-      {
-        float a0 = 0.f, a1 = 0.f;
-        if (hh == 1) { const float2 o = m->tot[pr]; a0 = o.x; a1 = o.y; }
-        const float gc0 = m->ref[4][c0], gc1 = m->ref[4][c0 + 1];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int t = 32 * hh + i;
-          float2 kv = make_float2(0.f, 0.f), qv = kv, gv = kv;
-          if (t < L) {
-            gv = bf2_to_f2(ld_u32(sm, OFF_G + sw128_off(t, c0, 8192)));
-            kv = bf2_to_f2(ld_u32(sm, OFF_K + sw128_off(t, c0, 8192)));
-            qv = bf2_to_f2(ld_u32(sm, OFF_Q + sw128_off(t, c0, 8192)));
+        for (int it = 0; it < 2; ++it) {
+          const int idx = tid + kCompute * it;
+          const int i = idx >> 3, oc = idx & 7;
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int jc = 8 * oc + e;
+            f[e] = (jc <= i) ? Tf[i * LDF + jc] * m->beta[jc] : 0.f;
           }
-          a0 += gv.x * kLog2e; a1 += gv.y * kLog2e;
-          const float e0 = ex2(a0), e1 = ex2(a1);
-          const float h0 = ex2(gc0 - a0), h1 = ex2(gc1 - a1);
-          const uint32_t off = sw128_off(t, c0, 8192);
-          st_u32(R, R_KT + off, f2_to_bf2(kv.x * e0, kv.y * e1));
-          st_u32(R, R_QT + off, f2_to_bf2(qv.x * e0, qv.y * e1));
-          st_u32(R, R_KH + off, f2_to_bf2(kv.x * h0, kv.y * h1));
+          at16(sm, OFF_TP + sw128_oct(i, oc, 8192)) = pack8(f);
         }
-        if (hh == 0) { m->ec[c0] = ex2(gc0); m->ec[c0 + 1] = ex2(gc1); }
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      sync_wg();
-      // q, k, g consumed: let the producer fetch the next chunk's tiles
-      if (tid == 0) mbar_arrive(&m->empty_qkg);
+      sync_for_mma();
       // ---------------------------------------------------------------- UMMA: W = T' Kt, U' = T' V
       if (tid == 0) wait_bounded(&m->full_v, par, m, limit, p.error_word);
       sync_wg();
@@ -469,147 +529,140 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid == 0) {
         tc_fence_after();
         const uint32_t id = idesc_bf16_f32(64, 128, 0, 1);
-        umma_k_loop(tmem + TM_WU, sm_u + OFF_R + R_TP, 16, true, 0, sm_u + OFF_R + R_KT, 8192, false, 0, 4, id,
+        umma_k_loop(tmem + TM_WU, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KT, 8192, false, 0, 4, id, false);
+        umma_k_loop(tmem + TM_WU + (16u << 16), sm_u + OFF_TP, 16, true, 0, sm_u + OFF_V, 8192, false, 0, 4, id,
                     false);
-        umma_k_loop(tmem + TM_WU + (16u << 16), sm_u + OFF_R + R_TP, 16, true, 0, sm_u + OFF_V, 8192, false, 0, 4,
-                    id, false);
       }
       if (!mma_commit_wait()) { ok = false; break; }
       if (tid == 0) mbar_arrive(&m->empty_v);
 
       // ---------------------------------------------------------------- -W -> bf16 (rows of the lane-0 tile)
       {
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
-        const int t = 16 * warp + lane;  // valid for lane < 16
+        const int t = 16 * q4 + lane;  // valid for lane < 16
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
+        for (int hb = 0; hb < 2; ++hb) {
+          const int c0 = wg * 64 + hb * 32;
           uint32_t v[32];
-          tmem_ld32(lane_base + TM_WU + 32 * cb, v);
+          tmem_ld32(tl + TM_WU + c0, v);
           tmem_wait_ld();
           if (lane < 16) {
 #pragma unroll
-            for (int jj = 0; jj < 32; jj += 2)
-              st_u32(R, R_W + sw128_off(t, 32 * cb + jj, 8192),
-                     f2_to_bf2(-__uint_as_float(v[jj]), -__uint_as_float(v[jj + 1])));
+            for (int oc = 0; oc < 4; ++oc) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) f[e] = -__uint_as_float(v[8 * oc + e]);
+              at16(sm, OFF_KT + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
+            }
           }
         }
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      sync_wg();
+      sync_for_mma();
       // ---------------------------------------------------------------- UMMA: U = U' - W S0 ; O = Qt S0
       if (tid == 0) {
         tc_fence_after();
         const uint32_t id = idesc_bf16_f32(64, 128, 0, 1);
-        umma_k_loop(tmem + TM_WU + (16u << 16), sm_u + OFF_R + R_W, 16, true, 8192, sm_u + OFF_S, 16384, false, 0,
-                    8, id, true);
-        umma_k_loop(tmem + TM_WU, sm_u + OFF_R + R_QT, 16, true, 8192, sm_u + OFF_S, 16384, false, 0, 8, id, false);
+        umma_k_loop(tmem + TM_WU + (16u << 16), sm_u + OFF_KT, 16, true, 8192, sm_u + OFF_S, 16384, false, 0, 8, id,
+                    true);
+        umma_k_loop(tmem + TM_WU, sm_u + OFF_QT, 16, true, 8192, sm_u + OFF_S, 16384, false, 0, 8, id, false);
       }
       if (!mma_commit_wait()) { ok = false; break; }
 
       // ---------------------------------------------------------------- U -> bf16 (rows of the lane-16 tile)
       {
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
-        const int t = 16 * warp + (lane - 16);  // valid for lane >= 16
+        const int t = 16 * q4 + lane - 16;  // valid for lane >= 16
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
+        for (int hb = 0; hb < 2; ++hb) {
+          const int c0 = wg * 64 + hb * 32;
           uint32_t v[32];
-          tmem_ld32(lane_base + TM_WU + 32 * cb, v);
+          tmem_ld32(tl + TM_WU + c0, v);
           tmem_wait_ld();
           if (lane >= 16) {
 #pragma unroll
-            for (int jj = 0; jj < 32; jj += 2)
-              st_u32(R, R_U + sw128_off(t, 32 * cb + jj, 8192),
-                     f2_to_bf2(__uint_as_float(v[jj]), __uint_as_float(v[jj + 1])));
-          }
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      sync_wg();
-      // ---------------------------------------------------------------- UMMA: O += P U ; K^T U
-      if (tid == 0) {
-        tc_fence_after();
-        umma_k_loop(tmem + TM_WU, sm_u + OFF_R + R_P, 16, true, 0, sm_u + OFF_R + R_U, 8192, false, 0, 4,
-                    idesc_bf16_f32(64, 128, 0, 1), true);
-        umma_k_loop(tmem + TM_KU, sm_u + OFF_R + R_KH, 8192, false, 0, sm_u + OFF_R + R_U, 8192, false, 0, 4,
-                    idesc_bf16_f32(128, 128, 1, 1), false);
-      }
-      if (!mma_commit_wait()) { ok = false; break; }
-
-      // ---------------------------------------------------------------- state carry
-      {
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
-        const float ec = m->ec[tid];
+            for (int oc = 0; oc < 4; ++oc) {
+              float f[8];
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-          uint32_t v[32];
-          tmem_ld32(lane_base + TM_KU + 32 * cb, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) S[32 * cb + jj] = ec * S[32 * cb + jj] + __uint_as_float(v[jj]);
-#pragma unroll
-          for (int jj = 0; jj < 32; jj += 2)
-            st_u32(sm, OFF_S + sw128_off(tid, 32 * cb + jj, 16384), f2_to_bf2(S[32 * cb + jj], S[32 * cb + jj + 1]));
-        }
-      }
-      // ---------------------------------------------------------------- epilogue
-      if (write_out) {
-        if (has_gate && tid == 0) wait_bounded(&m->full_gate, par, m, limit, p.error_word);
-        if (has_gate) sync_wg();
-        const bool gate_ok = *(volatile int32_t*)&m->abort == 0;
-        const uint32_t lane_base = tmem + ((uint32_t)(32 * warp) << 16);
-        const int t = 16 * warp + lane;  // O rows: lanes < 16
-        float ss = 0.f;
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-          uint32_t v[32];
-          tmem_ld32(lane_base + TM_WU + 32 * cb, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) { const float o = __uint_as_float(v[jj]) * p.scale; ss += o * o; }
-        }
-        const float rr = has_gate ? rsqrtf(ss / (float)DV + p.eps) : 1.f;
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + ((size_t)(tok + t) * H + h) * DV;
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-          uint32_t v[32];
-          tmem_ld32(lane_base + TM_WU + 32 * cb, v);
-          tmem_wait_ld();
-          if (lane < 16 && t < L && gate_ok) {
-#pragma unroll
-            for (int jj = 0; jj < 32; jj += 8) {
-              const int c = 32 * cb + jj;
-              float y[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(v[jj + e]) * p.scale * rr;
-              if (has_gate) {
-                const uint4 gq = *reinterpret_cast<const uint4*>(sm + OFF_GATE + sw128_off(t, c, 8192));
-                const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float2 gl = bf2_to_f2(gw[e]);
-                  const float w0 = p.norm_weight ? __ldg(p.norm_weight + c + 2 * e) : 1.f;
-                  const float w1 = p.norm_weight ? __ldg(p.norm_weight + c + 2 * e + 1) : 1.f;
-                  y[2 * e] *= w0 / (1.f + __expf(-gl.x));
-                  y[2 * e + 1] *= w1 / (1.f + __expf(-gl.y));
-                }
-              }
-              uint4 o;
-              o.x = f2_to_bf2(y[0], y[1]); o.y = f2_to_bf2(y[2], y[3]);
-              o.z = f2_to_bf2(y[4], y[5]); o.w = f2_to_bf2(y[6], y[7]);
-              *reinterpret_cast<uint4*>(orow + c) = o;
+              for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
+              at16(sm, OFF_KT + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
             }
           }
         }
-      } else if (has_gate) {
-        if (tid == 0) wait_bounded(&m->full_gate, par, m, limit, p.error_word);
       }
-      tc_fence_before();
-      sync_wg();
+      sync_for_mma();
+      // ---------------------------------------------------------------- UMMA: O += P U ; S += Kh^T U
+      if (tid == 0) {
+        tc_fence_after();
+        umma_k_loop(tmem + TM_WU, sm_u + OFF_P, 16, true, 0, sm_u + OFF_KT, 8192, false, 0, 4,
+                    idesc_bf16_f32(64, 128, 0, 1), true);
+        umma_k_loop(tmem + TM_S, sm_u + OFF_KH, 8192, false, 0, sm_u + OFF_KT, 8192, false, 0, 4,
+                    idesc_bf16_f32(128, 128, 1, 1), true);
+      }
+      if (!mma_commit_wait()) { ok = false; break; }
+
+      // ---------------------------------------------------------------- bf16 copy of the new state
+#pragma unroll
+      for (int hb = 0; hb < 2; ++hb) {
+        const int c0 = wg * 64 + hb * 32;
+        uint32_t v[32];
+        tmem_ld32(tl + TM_S + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int oc = 0; oc < 4; ++oc) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
+          at16(sm, OFF_S + sw128_oct(row, (c0 >> 3) + oc, 16384)) = pack8(f);
+        }
+      }
+      // ---------------------------------------------------------------- epilogue: RMSNorm * sigmoid(gate)
+      if (write_out) {
+        const int t = 16 * q4 + lane;  // O rows: lanes < 16
+        const bool act = lane < 16 && t < L;
+        const size_t orow = ((size_t)(tok + t) * H + h) * DV + wg * 64;
+        uint4 gq[8];
+        if (has_gate && act) {
+          const uint4* gp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.gate) + orow);
+#pragma unroll
+          for (int oc = 0; oc < 8; ++oc) gq[oc] = __ldg(gp + oc);
+        }
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tl + TM_WU + wg * 64, v0);
+        tmem_ld32(tl + TM_WU + wg * 64 + 32, v1);
+        tmem_wait_ld();
+        float ss = 0.f;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const float a0 = __uint_as_float(v0[jj]) * p.scale, a1 = __uint_as_float(v1[jj]) * p.scale;
+          ss += a0 * a0 + a1 * a1;
+        }
+        if (lane < 16) m->ss[wg][t] = ss;
+        sync_wg();
+        if (act) {
+          const float rr = has_gate ? rsqrtf((m->ss[0][t] + m->ss[1][t]) / (float)DV + p.eps) : 1.f;
+          const float sc = p.scale * rr;
+          uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow);
+#pragma unroll
+          for (int oc = 0; oc < 8; ++oc) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t u = oc < 4 ? v0[8 * oc + e] : v1[8 * (oc - 4) + e];
+              f[e] = __uint_as_float(u) * sc;
+            }
+            if (has_gate) {
+              float gl8[8];
+              unpack8(gq[oc], gl8);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float w = p.norm_weight ? __ldg(p.norm_weight + wg * 64 + 8 * oc + e) : 1.f;
+                f[e] *= __fdividef(w, 1.f + ex2(-gl8[e] * kLog2e));
+              }
+            }
+            op[oc] = pack8(f);
+          }
+        }
+      }
+      sync_for_mma();  // the bf16 state copy feeds the next chunk's UMMAs
       if (*(volatile int32_t*)&m->abort) { ok = false; break; }
-      if (tid == 0 && has_gate) mbar_arrive(&m->empty_gate);
-      fence_proxy_async_smem();  // the bf16 state copy feeds the next chunk's UMMAs
     }
 
     // ---------------------------------------------------------------- end state
@@ -622,8 +675,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (dst) {
 #pragma unroll
-        for (int c = 0; c < DV; c += 4)
-          *reinterpret_cast<float4*>(dst + (size_t)tid * DV + c) = make_float4(S[c], S[c + 1], S[c + 2], S[c + 3]);
+        for (int hb = 0; hb < 2; ++hb) {
+          const int c0 = wg * 64 + hb * 32;
+          uint32_t v[32];
+          tmem_ld32(tl + TM_S + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 32; jj += 4)
+            *reinterpret_cast<float4*>(dst + (size_t)row * DV + c0 + jj) =
+                make_float4(__uint_as_float(v[jj]), __uint_as_float(v[jj + 1]), __uint_as_float(v[jj + 2]),
+                            __uint_as_float(v[jj + 3]));
+        }
       }
     } else if (tid == 0 && mph > 0) {
       // an aborted UMMA group may still be running: wait for it before freeing TMEM
@@ -678,7 +740,6 @@ cudaError_t launch_chunk_tc(const Plan& plan, const ChunkParams& p, cudaStream_t
   if (!make_map(&maps.q, p.q, p.H, T) || !make_map(&maps.k, p.k, p.H, T) || !make_map(&maps.g, p.g, p.H, T) ||
       !make_map(&maps.v, p.v, p.H, T))
     return cudaErrorInvalidValue;
-  if (p.gate && !make_map(&maps.gate, p.gate, p.H, T)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
   chunk_tc_kernel<<<plan.n_seg * plan.H, kThreads, SMEM_BYTES, stream>>>(plan, maps, p);
