@@ -162,6 +162,7 @@ def dist_setup(n_gpus, backend="nccl"):
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's time: every rank's number is reduced with MAX."""
     if world == 1:
         return x
     import torch
@@ -169,6 +170,16 @@ def max_over_ranks(x: float, world: int, device) -> float:
     t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own batch (weak scaling: the work per GPU is fixed)."""
+    return base_seed + 1000 * rank
+
+
+def whole_job_rate(world: int, units_per_rank_step: float, steps: int, max_ms: float) -> float:
+    """Units processed by all ranks divided by the slowest rank's time."""
+    return world * units_per_rank_step * steps / (max_ms / 1e3)
 
 
 def barrier(world):
@@ -262,7 +273,7 @@ def run_ours(args):
 
     # ---------------- prefill workload (own batch per rank)
     w = synth.WORKLOADS[WORKLOAD]
-    inp = synth.make_workload(WORKLOAD, device=dev, seed=w["seed"] + 1000 * rank)
+    inp = synth.make_workload(WORKLOAD, device=dev, seed=rank_seed(w["seed"], rank))
     Bq, T, H, dk, dv = w["B"], w["T"], w["H"], w["dk"], w["dv"]
     out = torch.empty_like(inp.v)
     fin = torch.empty((Bq, H, dk, dv), dtype=torch.float32, device=dev)
@@ -309,7 +320,7 @@ def run_ours(args):
         raise RuntimeError(f"device error in timed region: {kda.kda_status_string(st)}")
 
     tokens_per_step = Bq * T
-    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
+    value = whole_job_rate(world, tokens_per_step, args.steps, elapsed_ms)
     head_tokens = Bq * T * H
     alg_bytes = head_tokens * BYTES_PER_HEAD_TOKEN + Bq * H * STATE_BYTES  # final states written
     alg_flops = head_tokens * FLOPS_PER_HEAD_TOKEN
@@ -409,7 +420,7 @@ def run_decode(args, dev, stream, rank, world, peaks, peak_src, clocks):
     from linear_attention_serving_rule_b200 import synth
     w = synth.WORKLOADS[DECODE]
     N, H, dk, dv, ring = w["N"], w["H"], w["dk"], w["dv"], w["ring"]
-    seed = w["seed"] + 1000 * rank
+    seed = rank_seed(w["seed"], rank)
     state = synth.make_states(slots=N, H=H, dk=dk, dv=dv, seed=seed, device=dev)
     toks = [synth.make_decode_token(N=N, H=H, dk=dk, dv=dv, seed=seed + 1 + i, device=dev)
             for i in range(ring)]

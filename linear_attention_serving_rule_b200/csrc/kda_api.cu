@@ -200,15 +200,23 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
     for (int32_t q = 0; q < np; ++q) {
       const int32_t t0 = sp.tok0 + q * sl;
       const int32_t len = std::min(sl, sp.len - q * sl);
-      if (q == 0) head.push_back({t0, len, sp.seq, kRoleHead, b, 0});
-      else if (q < np - 1) local.push_back({t0, len, sp.seq, kRoleLocal, b + q, 0});
+      if (q == 0) {
+        head.push_back({t0, len, sp.seq, kRoleHead, b, 0});
+      } else if (q < np - 1) {
+        if (use_tc) {  // S_loc and M as two plain-state units of the tensor-core kernel
+          local.push_back({t0, len, sp.seq, kRoleLocalS, b + q, 0});
+          local.push_back({t0, len, sp.seq, kRoleLocalM, b + q, 0});
+        } else {
+          local.push_back({t0, len, sp.seq, kRoleLocal, b + q, 0});
+        }
+      }
       if (q == 0) whole.push_back({t0, len, sp.seq, kRoleWhole, b, 0});
       else whole.push_back({t0, len, sp.seq, kRoleFromWs, b + q, q == np - 1 ? 1 : 0});
     }
   }
   cudaError_t e = cudaSuccess;
   if (!head.empty()) e = run_segments(head, p, a->dtype, use_tc, stream);
-  if (e == cudaSuccess && !local.empty()) e = run_segments(local, p, a->dtype, false, stream);
+  if (e == cudaSuccess && !local.empty()) e = run_segments(local, p, a->dtype, use_tc, stream);
   if (e == cudaSuccess && L.any_split) {
     // combine: S_start(q+1) = M_q S_start(q) + S_loc(q), sequential over q per (sequence, head)
     static thread_local Plan plan;

@@ -54,20 +54,20 @@ constexpr int kThreads = 288;
 constexpr float kLog2e = 1.4426950408889634f;
 
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_KQ = 0;       // k rows 0-63 | q rows 64-127 (TMA), then [k; q] e^{gamma - r_own} in place
+constexpr uint32_t OFF_KQ = 0;       // k rows 0-63 | q rows 64-127 (TMA); later e^{gamma} k | e^{gamma} q in place
 constexpr uint32_t OFF_G = 32768;    // g (TMA)
 constexpr uint32_t OFF_V = 49152;    // v (TMA), B operand of U' = T' V
 constexpr uint32_t OFF_KC = 65536;   // Kc_0..Kc_3 (40 KB); then fp32 A and T of the inverse
-constexpr uint32_t OFF_KT = 106496;  // e^{gamma} k; then -W; then U
-constexpr uint32_t OFF_QT = 122880;  // e^{gamma} q
+constexpr uint32_t OFF_KL = 106496;  // [k; q] e^{gamma - r_own} (128 rows, 32 KB); then -W; then U
 constexpr uint32_t OFF_KH = 139264;  // e^{gamma_C - gamma} k
 constexpr uint32_t OFF_S = 155648;   // bf16 state, MN-major [dk rows][dv], two 16 KB column blocks
 constexpr uint32_t OFF_TP = 188416;  // T' = T Diag(beta), bf16 [64][64]
 constexpr uint32_t OFF_P = 196608;   // P (causally masked), bf16 [64][64]
 constexpr uint32_t OFF_MISC = 204800;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 8192 + 1024;
-constexpr uint32_t OFF_TF = OFF_KC + 16640;  // fp32 T, after fp32 A (both [64][65])
-constexpr int LDF = 65;
+constexpr uint32_t OFF_TF = OFF_KC + 16640;  // fp32 T [64][68], after fp32 A [64][65]
+constexpr int LDF = 65;  // row stride of A (scalar column writes, conflict-free)
+constexpr int LDT = 68;  // row stride of T (16-byte aligned rows for float4 access)
 
 constexpr uint32_t TM_S = 0, TM_AP = 128, TM_WU = 288;
 
@@ -80,7 +80,7 @@ struct Misc {
   uint64_t full_qkg, full_v, empty_qkg, empty_v, mma;
   uint32_t tmem_base;
   int32_t abort;
-  float beta[C];
+  float beta[2][C];  // double-buffered by chunk parity (written by the producer warp)
   float se[4][DK];  // e^{decay over sub-tile m}, per channel
   float ec[DK];     // e^{gamma_C}
   float ss[2][C];   // epilogue: partial sums of squares of the two column halves
@@ -166,6 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t limit = (p.flags & KDA_FLAG_TEST_FORCE_TIMEOUT) ? 0ull : 2000000000ull;  // 2 s
   const uint64_t drain_limit = 2000000000ull;
   const int nchunks = (seg.len + C - 1) / C;
+  const bool need_v = seg.role != kRoleLocalM;  // the transition pass runs with values = 0
 
   if (tid == 0) {
     mbar_init(&m->full_qkg, 1); mbar_init(&m->full_v, 1);
@@ -188,29 +189,46 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 8) {
     // ===================================================================== TMA producer
-    if (lane == 0) {
-      int iq = -1, iv = -1;  // last chunk whose q/k/g and v loads were issued
-      for (int j = 0; j < nchunks; ++j) {
-        const int32_t tok = seg.tok0 + j * C;
-        const uint32_t par = (uint32_t)((j & 1) ^ 1);
-        if (!wait_bounded(&m->empty_qkg, par, m, drain_limit, p.error_word)) break;
+    // Lane 0 issues the tile loads; the whole warp first fetches the chunk's beta into the
+    // double buffer m->beta[j & 1] (published by the same mbarrier as the q/k/g tiles).
+    int iq = -1, iv = -1;  // last chunk whose q/k/g and v loads were issued
+    for (int j = 0; j < nchunks; ++j) {
+      const int32_t tok = seg.tok0 + j * C;
+      const int L = min(C, seg.len - j * C);
+      const uint32_t par = (uint32_t)((j & 1) ^ 1);
+      int okw = 1;
+      if (lane == 0) okw = wait_bounded(&m->empty_qkg, par, m, drain_limit, p.error_word) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (!okw) break;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int t = lane + 32 * r;
+        m->beta[j & 1][t] = (t < L) ? to_f32(static_cast<const __nv_bfloat16*>(p.beta)[(size_t)(tok + t) * H + h]) : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) {
         mbar_arrive_expect_tx(&m->full_qkg, 3 * 16384);
         for (int hf = 0; hf < 2; ++hf) {
           tma_load_3d(sm + OFF_KQ + hf * 16384, &maps.k, &m->full_qkg, hf * 64, h, tok);
           tma_load_3d(sm + OFF_KQ + hf * 16384 + 8192, &maps.q, &m->full_qkg, hf * 64, h, tok);
           tma_load_3d(sm + OFF_G + hf * 8192, &maps.g, &m->full_qkg, hf * 64, h, tok);
         }
-        iq = j;
-        if (!wait_bounded(&m->empty_v, par, m, drain_limit, p.error_word)) break;
+      }
+      iq = j;
+      if (!need_v) continue;
+      if (lane == 0) okw = wait_bounded(&m->empty_v, par, m, drain_limit, p.error_word) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (!okw) break;
+      if (lane == 0) {
         mbar_arrive_expect_tx(&m->full_v, 16384);
         for (int hf = 0; hf < 2; ++hf) tma_load_3d(sm + OFF_V + hf * 8192, &maps.v, &m->full_v, hf * 64, h, tok);
-        iv = j;
       }
-      // drain: after an abort, wait (bounded, regardless of the abort) for the loads issued
-      if (*(volatile int32_t*)&m->abort) {
-        if (iq >= 0) wait_bounded(&m->full_qkg, (uint32_t)(iq & 1), m, drain_limit, p.error_word, false);
-        if (iv >= 0) wait_bounded(&m->full_v, (uint32_t)(iv & 1), m, drain_limit, p.error_word, false);
-      }
+      iv = j;
+    }
+    // drain: after an abort, wait (bounded, regardless of the abort) for the loads issued
+    if (lane == 0 && *(volatile int32_t*)&m->abort) {
+      if (iq >= 0) wait_bounded(&m->full_qkg, (uint32_t)(iq & 1), m, drain_limit, p.error_word, false);
+      if (iv >= 0) wait_bounded(&m->full_v, (uint32_t)(iv & 1), m, drain_limit, p.error_word, false);
     }
   } else {
     // ===================================================================== compute warpgroups
@@ -251,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (seg.role == kRoleFromWs) {
         src = p.ws_state + ((size_t)seg.slot * H + h) * unit_state;
       }
+      const bool ident = seg.role == kRoleLocalM;  // transition pass: start from I
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
         const int c0 = wg * 64 + hb * 32;
@@ -261,6 +280,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                          : make_float4(0.f, 0.f, 0.f, 0.f);
           v[jj] = __float_as_uint(x.x); v[jj + 1] = __float_as_uint(x.y);
           v[jj + 2] = __float_as_uint(x.z); v[jj + 3] = __float_as_uint(x.w);
+        }
+        if (ident) {
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) v[jj] = __float_as_uint(c0 + jj == row ? 1.f : 0.f);
         }
         tmem_st32(tl + TM_S + c0, v);
 #pragma unroll
@@ -274,23 +297,90 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
     }
 
+    // Epilogue of one chunk: O sits at TMEM lane offset 0 of [288,416) until the next chunk's
+    // W/U' UMMAs, so it runs in the shadow of the next chunk's Gram UMMAs.  Lanes < 16 of each
+    // warp hold the 64 O rows; the two warpgroups hold the two column halves and exchange their
+    // partial sums of squares; the gate logits come from the staging copy made by load_gate.
+    // The gate logits of a chunk are staged with cp.async into the T'/P region, which is free from
+    // the start of the next chunk until its Gram read-out; row t at OFF_TP + 256 t, 16-byte chunk c
+    // at position c ^ (t & 15).
+    auto load_gate = [&](int L_e, int32_t tok_e) {
+      if (!has_gate) return;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int idx = tid + kCompute * r;
+        const int t = idx >> 4, c16 = idx & 15;
+        if (t < L_e)
+          cp_async_16(sm_u + OFF_TP + t * 256 + ((c16 ^ (t & 15)) << 4),
+                      static_cast<const __nv_bfloat16*>(p.gate) + ((size_t)(tok_e + t) * H + h) * DV + 8 * c16);
+      }
+      cp_async_commit();
+    };
+    auto epilogue = [&](int L_e, int32_t tok_e) {
+      const int t = 16 * q4 + lane;
+      const bool act = lane < 16 && t < L_e;
+      float ss = 0.f;
+#pragma unroll
+      for (int hb = 0; hb < 2; ++hb) {
+        uint32_t v[32];
+        tmem_ld32(tl + TM_WU + wg * 64 + 32 * hb, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const float a = __uint_as_float(v[jj]) * p.scale;
+          ss += a * a;
+        }
+      }
+      if (lane < 16) m->ss[wg][t] = ss;
+      cp_async_wait_all();
+      sync_wg();
+      const float rr = (has_gate && lane < 16) ? rsqrtf((m->ss[0][t] + m->ss[1][t]) / (float)DV + p.eps) : 1.f;
+      const float sc = p.scale * rr;
+      uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ((size_t)(tok_e + t) * H + h) * DV +
+                                           wg * 64);
+#pragma unroll
+      for (int hb = 0; hb < 2; ++hb) {
+        uint32_t v[32];
+        tmem_ld32(tl + TM_WU + wg * 64 + 32 * hb, v);
+        tmem_wait_ld();
+        if (act) {
+#pragma unroll
+          for (int oc = 0; oc < 4; ++oc) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]) * sc;
+            if (has_gate) {
+              float gl8[8];
+              const int c16 = wg * 8 + 4 * hb + oc;
+              unpack8(at16(sm, OFF_TP + t * 256 + ((c16 ^ (t & 15)) << 4)), gl8);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float w = p.norm_weight ? __ldg(p.norm_weight + wg * 64 + 32 * hb + 8 * oc + e) : 1.f;
+                f[e] *= __fdividef(w, 1.f + ex2(-gl8[e] * kLog2e));
+              }
+            }
+            op[4 * hb + oc] = pack8(f);
+          }
+        }
+      }
+    };
+
+    int L_prev = 0;
+    int32_t tok_prev = 0;
     for (int j = 0; j < nchunks && ok; ++j) {
       const int L = min(C, seg.len - j * C);
       const int32_t tok = seg.tok0 + j * C;
       const uint32_t par = (uint32_t)(j & 1);
-      if (tid < C) {
-        float b = 0.f;
-        if (tid < L) b = to_f32(static_cast<const __nv_bfloat16*>(p.beta)[(size_t)(tok + tid) * H + h]);
-        m->beta[tid] = b;
-      }
+      const float* beta = m->beta[j & 1];
+      if (write_out && j > 0) load_gate(L_prev, tok_prev);  // consumed by its epilogue below
       if (!wg_wait(&m->full_qkg, par)) { ok = false; break; }
 
-      // ---------------------------------------------------------------- decay prep (one pass)
+      // ---------------------------------------------------------------- decay prep A: Gram operands
       // thread: channels 8o .. 8o+7, tokens t0 .. t0+3 of sub-tile b
+      const int qq = tid & 3, o = (tid >> 2) & 15, b = tid >> 6;
+      const int t0 = 16 * b + 4 * qq;
+      float gl[4][8];     // inclusive cumulative log2-decay from the sub-tile start
       {
-        const int qq = tid & 3, o = (tid >> 2) & 15, b = tid >> 6;
-        const int t0 = 16 * b + 4 * qq;
-        float gl[4][8];  // inclusive cumulative log2-decay from the sub-tile start
         float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -324,34 +414,37 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 4; ++i) gl[i][e] += excl;
           if (qq == 3) m->se[b][8 * o + e] = ex2(x);  // decay over the whole sub-tile
         }
-        sync_wg();
-        // Per-channel factors, split so that no product of an O(1) value with an underflowed
-        // factor is lost: with se_m = e^{decay over sub-tile m},
-        //   Eb   = e^{r_b}                       = prod_{m<b} se_m
-        //   Rh_a = e^{r_a - r_{b+1}}  (a > b)    = prod_{b<m<a} se_m
-        //   Ehi  = e^{gamma_C - r_{b+1}}         = prod_{m>b} se_m
-        // and per token ix * se_b = e^{r_{b+1} - gamma_t} lies in [e^-80, 1].
-        float Eb[8], Ehi[8], sb[8], Rh[4][8];
+      }
+      sync_wg();
+      // Per-channel factors, split so that no product of an O(1) value with an underflowed
+      // factor is lost: with se_m = e^{decay over sub-tile m},
+      //   Eb   = e^{r_b}                       = prod_{m<b} se_m
+      //   Rh_a = e^{r_a - r_{b+1}}  (a > b)    = prod_{b<m<a} se_m
+      //   Ehi  = e^{gamma_C - r_{b+1}}         = prod_{m>b} se_m
+      // and per token ix * se_b = e^{r_{b+1} - gamma_t} lies in [e^-80, 1].
+      float Eb[8], Ehi[8], sb[8];
+      {
+        float s1[8], s2[8];  // se_{b+1}, se_{b+2} (1 past the last sub-tile)
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           float se[4];
 #pragma unroll
           for (int mm = 0; mm < 4; ++mm) se[mm] = m->se[mm][8 * o + e];
-          float eb = 1.f, ehi = 1.f, r = 1.f;
+          float eb = 1.f, ehi = 1.f;
 #pragma unroll
           for (int mm = 0; mm < 4; ++mm) {
             if (mm < b) eb *= se[mm];
             if (mm > b) ehi *= se[mm];
-            Rh[mm][e] = r;  // for mm > b: prod over b < m < mm
-            if (mm > b) r *= se[mm];
           }
           Eb[e] = eb; Ehi[e] = ehi;
           sb[e] = b == 0 ? se[0] : b == 1 ? se[1] : b == 2 ? se[2] : se[3];
+          s1[e] = b == 0 ? se[1] : b == 1 ? se[2] : b == 2 ? se[3] : 1.f;
+          s2[e] = b == 0 ? se[2] : b == 1 ? se[3] : 1.f;
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int t = t0 + i;
-          float kf[8], qf[8];
+          float kf[8], qf[8], x[8], ix[8], f[8];
           if (t < L) {
             unpack8(at16(sm, OFF_KQ + sw128_oct(t, o, 16384)), kf);
             unpack8(at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)), qf);
@@ -359,31 +452,31 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) { kf[e] = 0.f; qf[e] = 0.f; }
           }
-          float x[8], ix[8], ixs[8], f[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) { x[e] = ex2(gl[i][e]); ix[e] = ex2(-gl[i][e]); ixs[e] = ix[e] * sb[e]; }
-          const uint32_t o64 = sw128_oct(t, o, 8192);
+          for (int e = 0; e < 8; ++e) { x[e] = ex2(gl[i][e]); ix[e] = ex2(-gl[i][e]); }
 #pragma unroll
           for (int e = 0; e < 8; ++e) f[e] = kf[e] * x[e];
-          at16(sm, OFF_KQ + sw128_oct(t, o, 16384)) = pack8(f);
+          at16(sm, OFF_KL + sw128_oct(t, o, 16384)) = pack8(f);
 #pragma unroll
           for (int e = 0; e < 8; ++e) f[e] = qf[e] * x[e];
-          at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)) = pack8(f);
+          at16(sm, OFF_KL + sw128_oct(64 + t, o, 16384)) = pack8(f);
+          // Kc_a = k e^{r_a - gamma_t}: k ix for a = b, then k ix se_b se_{b+1} ... se_{a-1}
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = kf[e] * x[e] * Eb[e];
-          at16(sm, OFF_KT + o64) = pack8(f);
+          for (int e = 0; e < 8; ++e) f[e] = kf[e] * ix[e];
+          at16(sm, OFF_KC + kc_off(b) + sw128_oct(t, o, 2048u * (b + 1))) = pack8(f);
+          if (b < 3) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = qf[e] * x[e] * Eb[e];
-          at16(sm, OFF_QT + o64) = pack8(f);
+            for (int e = 0; e < 8; ++e) f[e] = kf[e] * ix[e] * sb[e];
+            at16(sm, OFF_KC + kc_off(b + 1) + sw128_oct(t, o, 2048u * (b + 2))) = pack8(f);
+            if (b < 2) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = kf[e] * ixs[e] * Ehi[e];
-          at16(sm, OFF_KH + o64) = pack8(f);
+              for (int e = 0; e < 8; ++e) f[e] *= s1[e];
+              at16(sm, OFF_KC + kc_off(b + 2) + sw128_oct(t, o, 2048u * (b + 3))) = pack8(f);
+              if (b < 1) {
 #pragma unroll
-          for (int a = 0; a < 4; ++a) {
-            if (a >= b) {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) f[e] = (a == b) ? kf[e] * ix[e] : kf[e] * ixs[e] * Rh[a][e];
-              at16(sm, OFF_KC + kc_off(a) + sw128_oct(t, o, 2048u * (a + 1))) = pack8(f);
+                for (int e = 0; e < 8; ++e) f[e] *= s2[e];
+                at16(sm, OFF_KC + kc_off(3) + sw128_oct(t, o, 8192u)) = pack8(f);
+              }
             }
           }
         }
@@ -396,23 +489,58 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int a = 0; a < 4; ++a) {
           const uint32_t n = 16u * (a + 1);
-          umma_k_loop(tmem + TM_AP + ap_off(a), sm_u + OFF_KQ, 16, true, 16384, sm_u + OFF_KC + kc_off(a), 16, true,
+          umma_k_loop(tmem + TM_AP + ap_off(a), sm_u + OFF_KL, 16, true, 16384, sm_u + OFF_KC + kc_off(a), 16, true,
                       n * 128u, 8, idesc_bf16_f32(128, n, 0, 0), false);
         }
         umma_commit(&m->mma);
       }
-      // while the Gram UMMAs run: decay the fp32 state in place, S <- Diag(e^{gamma_C}) S
+      // ---------------------------------------------------------------- in the shadow of the Gram UMMAs:
+      // (1) decay prep B, in place over the raw tiles: e^{gamma} k over k, e^{gamma} q over q,
+      //     and e^{gamma_C - gamma} k
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = t0 + i;
+        float kf[8], qf[8], x[8], f[8];
+        if (t < L) {
+          unpack8(at16(sm, OFF_KQ + sw128_oct(t, o, 16384)), kf);
+          unpack8(at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)), qf);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) { kf[e] = 0.f; qf[e] = 0.f; }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = ex2(gl[i][e]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = kf[e] * x[e] * Eb[e];
+        at16(sm, OFF_KQ + sw128_oct(t, o, 16384)) = pack8(f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = qf[e] * x[e] * Eb[e];
+        at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)) = pack8(f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = kf[e] * ex2(-gl[i][e]) * sb[e] * Ehi[e];
+        at16(sm, OFF_KH + sw128_oct(t, o, 8192)) = pack8(f);
+      }
+      // (2) the previous chunk's epilogue (its O is still in TMEM)
+      if (write_out && j > 0) epilogue(L_prev, tok_prev);
+      // (3) bf16 copy of the chunk's start state for the UMMAs, then S <- Diag(e^{gamma_C}) S in place
       {
         const float ec = m->ec[row];
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
-          const uint32_t col = TM_S + wg * 64 + hb * 32;
+          const int c0 = wg * 64 + hb * 32;
           uint32_t v[32];
-          tmem_ld32(tl + col, v);
+          tmem_ld32(tl + TM_S + c0, v);
           tmem_wait_ld();
 #pragma unroll
+          for (int oc = 0; oc < 4; ++oc) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
+            at16(sm, OFF_S + sw128_oct(row, (c0 >> 3) + oc, 16384)) = pack8(f);
+          }
+#pragma unroll
           for (int jj = 0; jj < 32; ++jj) v[jj] = __float_as_uint(__uint_as_float(v[jj]) * ec);
-          tmem_st32(tl + col, v);
+          tmem_st32(tl + TM_S + c0, v);
         }
         tmem_wait_st();
       }
@@ -422,7 +550,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (!r) { ok = false; break; }
       }
-      if (tid == 0) mbar_arrive(&m->empty_qkg);  // k, q, g fully consumed
 
       // ---------------------------------------------------------------- read A (beta-scaled) and P
       {
@@ -431,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t = (q4 & 1) * 32 + lane;
         const int a = 2 * (q4 & 1) + wg;  // the sub-tile whose columns this warp loads
         const bool mine = (t >> 4) == a;
-        const float bt = m->beta[t];
+        const float bt = beta[t];
 #pragma unroll
         for (int kb = 0; kb < 4; ++kb) {
           if (kb <= a) {
@@ -464,47 +591,66 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       sync_wg();
-
       // ---------------------------------------------------------------- UT inverse: T' = (I + Diag(beta) A)^-1 Diag(beta)
+      // L = Diag(beta) A (strictly lower).  Diagonal 16x16 blocks of T by forward substitution
+      // (one column per thread), then the off-diagonal blocks by block distance d:
+      //   T_ab = -T_aa sum_{c in blocks b..a-1} L_{a c} T_{c b},  a = b + d.
       {
         const float* Lf = reinterpret_cast<const float*>(sm + OFF_KC);
         float* Tf = reinterpret_cast<float*>(sm + OFF_TF);
         float* Y = m->y;
-        if (tid < 64) {  // diagonal 16x16 blocks by forward substitution, one column per thread
+        if (tid < 64) {
           const int a = tid >> 4, jc = tid & 15, o = 16 * a;
           float col[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) col[i] = (i == jc) ? 1.f : 0.f;
 #pragma unroll
           for (int i = 1; i < 16; ++i) {
-            if (i > jc) {
-              float acc = 0.f;
+            const float* lr = Lf + (o + i) * LDF + o;
+            float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-              for (int mm = 0; mm < 15; ++mm)
-                if (mm < i && mm >= jc) acc += Lf[(o + i) * LDF + o + mm] * col[mm];
-              col[i] = -acc;
-            }
+            for (int mm = 0; mm < i; ++mm) s4[mm & 3] += lr[mm] * col[mm];  // col[mm] = 0 for mm < jc
+            const float acc = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+            col[i] = (i == jc) ? 1.f : (i > jc ? -acc : 0.f);
           }
 #pragma unroll
-          for (int i = 0; i < 16; ++i) Tf[(o + i) * LDF + o + jc] = col[i];
+          for (int i = 0; i < 16; ++i) Tf[(o + i) * LDT + o + jc] = col[i];
         }
         sync_wg();
-        for (int d = 1; d <= 3; ++d) {  // off-diagonal blocks at block distance d
-          const int nel = (4 - d) * 256;
-          for (int e = tid; e < nel; e += kCompute) {
-            const int b = e >> 8, i = (e >> 4) & 15, jc = e & 15, a = b + d;
-            const float* lrow = Lf + (16 * a + i) * LDF;
-            float acc = 0.f;
-            for (int cc = 16 * b; cc < 16 * a; ++cc) acc += lrow[cc] * Tf[cc * LDF + 16 * b + jc];
-            Y[e] = acc;
+#pragma unroll
+        for (int d = 1; d <= 3; ++d) {
+          const int nstrip = (4 - d) * 64;  // (block, row, 4-column strip)
+          const int b = tid >> 6, i = (tid >> 2) & 15, j0 = (tid & 3) * 4, a = b + d;
+          if (tid < nstrip) {  // Y = L_{a, blocks b..a-1} T_{blocks b..a-1, b}
+            const float* lrow = Lf + (16 * a + i) * LDF + 16 * b;
+            const float* tcol = Tf + 16 * b * LDT + 16 * b + j0;
+            float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+#pragma unroll
+            for (int cc = 0; cc < 16 * d; cc += 2) {
+              const float l0 = lrow[cc], l1 = lrow[cc + 1];
+              const float4 t0v = *reinterpret_cast<const float4*>(tcol + cc * LDT);
+              const float4 t1v = *reinterpret_cast<const float4*>(tcol + (cc + 1) * LDT);
+              acc0.x += l0 * t0v.x; acc0.y += l0 * t0v.y; acc0.z += l0 * t0v.z; acc0.w += l0 * t0v.w;
+              acc1.x += l1 * t1v.x; acc1.y += l1 * t1v.y; acc1.z += l1 * t1v.z; acc1.w += l1 * t1v.w;
+            }
+            *reinterpret_cast<float4*>(Y + 4 * tid) =
+                make_float4(acc0.x + acc1.x, acc0.y + acc1.y, acc0.z + acc1.z, acc0.w + acc1.w);
           }
           sync_wg();
-          for (int e = tid; e < nel; e += kCompute) {
-            const int b = e >> 8, i = (e >> 4) & 15, jc = e & 15, a = b + d;
-            const float* trow = Tf + (16 * a + i) * LDF + 16 * a;
-            float acc = 0.f;
-            for (int kk = 0; kk <= i; ++kk) acc += trow[kk] * Y[(b << 8) + (kk << 4) + jc];
-            Tf[(16 * a + i) * LDF + 16 * b + jc] = -acc;
+          if (tid < nstrip) {  // T_ab = -T_aa Y  (T_aa is lower triangular with exact zeros above)
+            const float* trow = Tf + (16 * a + i) * LDT + 16 * a;
+            const float* ycol = Y + (b * 16) * 16 + j0;
+            float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+#pragma unroll
+            for (int kk = 0; kk < 16; kk += 2) {
+              const float u0 = trow[kk], u1 = trow[kk + 1];
+              const float4 y0 = *reinterpret_cast<const float4*>(ycol + kk * 16);
+              const float4 y1 = *reinterpret_cast<const float4*>(ycol + (kk + 1) * 16);
+              acc0.x += u0 * y0.x; acc0.y += u0 * y0.y; acc0.z += u0 * y0.z; acc0.w += u0 * y0.w;
+              acc1.x += u1 * y1.x; acc1.y += u1 * y1.y; acc1.z += u1 * y1.z; acc1.w += u1 * y1.w;
+            }
+            *reinterpret_cast<float4*>(Tf + (16 * a + i) * LDT + 16 * b + j0) =
+                make_float4(-(acc0.x + acc1.x), -(acc0.y + acc1.y), -(acc0.z + acc1.z), -(acc0.w + acc1.w));
           }
           sync_wg();
         }
@@ -512,29 +658,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int it = 0; it < 2; ++it) {
           const int idx = tid + kCompute * it;
           const int i = idx >> 3, oc = idx & 7;
+          const float4 t0 = *reinterpret_cast<const float4*>(Tf + i * LDT + 8 * oc);
+          const float4 t1 = *reinterpret_cast<const float4*>(Tf + i * LDT + 8 * oc + 4);
+          const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
           float f[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int jc = 8 * oc + e;
-            f[e] = (jc <= i) ? Tf[i * LDF + jc] * m->beta[jc] : 0.f;
+            f[e] = (jc <= i) ? tv[e] * beta[jc] : 0.f;
           }
           at16(sm, OFF_TP + sw128_oct(i, oc, 8192)) = pack8(f);
         }
       }
       sync_for_mma();
       // ---------------------------------------------------------------- UMMA: W = T' Kt, U' = T' V
-      if (tid == 0) wait_bounded(&m->full_v, par, m, limit, p.error_word);
+      if (tid == 0 && need_v) wait_bounded(&m->full_v, par, m, limit, p.error_word);
       sync_wg();
       if (*(volatile int32_t*)&m->abort) { ok = false; break; }
       if (tid == 0) {
         tc_fence_after();
         const uint32_t id = idesc_bf16_f32(64, 128, 0, 1);
-        umma_k_loop(tmem + TM_WU, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KT, 8192, false, 0, 4, id, false);
-        umma_k_loop(tmem + TM_WU + (16u << 16), sm_u + OFF_TP, 16, true, 0, sm_u + OFF_V, 8192, false, 0, 4, id,
-                    false);
+        umma_k_loop(tmem + TM_WU, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ, 16384, false, 0, 4, id, false);
+        if (need_v)
+          umma_k_loop(tmem + TM_WU + (16u << 16), sm_u + OFF_TP, 16, true, 0, sm_u + OFF_V, 8192, false, 0, 4, id,
+                      false);
       }
       if (!mma_commit_wait()) { ok = false; break; }
-      if (tid == 0) mbar_arrive(&m->empty_v);
+      if (tid == 0 && need_v) mbar_arrive(&m->empty_v);
 
       // ---------------------------------------------------------------- -W -> bf16 (rows of the lane-0 tile)
       {
@@ -551,7 +701,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               float f[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) f[e] = -__uint_as_float(v[8 * oc + e]);
-              at16(sm, OFF_KT + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
+              at16(sm, OFF_KL + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
             }
           }
         }
@@ -561,11 +711,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid == 0) {
         tc_fence_after();
         const uint32_t id = idesc_bf16_f32(64, 128, 0, 1);
-        umma_k_loop(tmem + TM_WU + (16u << 16), sm_u + OFF_KT, 16, true, 8192, sm_u + OFF_S, 16384, false, 0, 8, id,
-                    true);
-        umma_k_loop(tmem + TM_WU, sm_u + OFF_QT, 16, true, 8192, sm_u + OFF_S, 16384, false, 0, 8, id, false);
+        umma_k_loop(tmem + TM_WU + (16u << 16), sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S, 16384, false, 0, 8, id,
+                    need_v);
+        umma_k_loop(tmem + TM_WU, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S, 16384, false, 0, 8, id, false);
       }
       if (!mma_commit_wait()) { ok = false; break; }
+      if (tid == 0) mbar_arrive(&m->empty_qkg);  // k, q, g and their in-place products consumed
 
       // ---------------------------------------------------------------- U -> bf16 (rows of the lane-16 tile)
       {
@@ -582,7 +733,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               float f[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
-              at16(sm, OFF_KT + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
+              at16(sm, OFF_KL + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
             }
           }
         }
@@ -591,78 +742,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------------- UMMA: O += P U ; S += Kh^T U
       if (tid == 0) {
         tc_fence_after();
-        umma_k_loop(tmem + TM_WU, sm_u + OFF_P, 16, true, 0, sm_u + OFF_KT, 8192, false, 0, 4,
+        umma_k_loop(tmem + TM_WU, sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL, 8192, false, 0, 4,
                     idesc_bf16_f32(64, 128, 0, 1), true);
-        umma_k_loop(tmem + TM_S, sm_u + OFF_KH, 8192, false, 0, sm_u + OFF_KT, 8192, false, 0, 4,
+        umma_k_loop(tmem + TM_S, sm_u + OFF_KH, 8192, false, 0, sm_u + OFF_KL, 8192, false, 0, 4,
                     idesc_bf16_f32(128, 128, 1, 1), true);
       }
       if (!mma_commit_wait()) { ok = false; break; }
 
-      // ---------------------------------------------------------------- bf16 copy of the new state
-#pragma unroll
-      for (int hb = 0; hb < 2; ++hb) {
-        const int c0 = wg * 64 + hb * 32;
-        uint32_t v[32];
-        tmem_ld32(tl + TM_S + c0, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int oc = 0; oc < 4; ++oc) {
-          float f[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
-          at16(sm, OFF_S + sw128_oct(row, (c0 >> 3) + oc, 16384)) = pack8(f);
-        }
-      }
-      // ---------------------------------------------------------------- epilogue: RMSNorm * sigmoid(gate)
-      if (write_out) {
-        const int t = 16 * q4 + lane;  // O rows: lanes < 16
-        const bool act = lane < 16 && t < L;
-        const size_t orow = ((size_t)(tok + t) * H + h) * DV + wg * 64;
-        uint4 gq[8];
-        if (has_gate && act) {
-          const uint4* gp = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.gate) + orow);
-#pragma unroll
-          for (int oc = 0; oc < 8; ++oc) gq[oc] = __ldg(gp + oc);
-        }
-        uint32_t v0[32], v1[32];
-        tmem_ld32(tl + TM_WU + wg * 64, v0);
-        tmem_ld32(tl + TM_WU + wg * 64 + 32, v1);
-        tmem_wait_ld();
-        float ss = 0.f;
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const float a0 = __uint_as_float(v0[jj]) * p.scale, a1 = __uint_as_float(v1[jj]) * p.scale;
-          ss += a0 * a0 + a1 * a1;
-        }
-        if (lane < 16) m->ss[wg][t] = ss;
-        sync_wg();
-        if (act) {
-          const float rr = has_gate ? rsqrtf((m->ss[0][t] + m->ss[1][t]) / (float)DV + p.eps) : 1.f;
-          const float sc = p.scale * rr;
-          uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow);
-#pragma unroll
-          for (int oc = 0; oc < 8; ++oc) {
-            float f[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint32_t u = oc < 4 ? v0[8 * oc + e] : v1[8 * (oc - 4) + e];
-              f[e] = __uint_as_float(u) * sc;
-            }
-            if (has_gate) {
-              float gl8[8];
-              unpack8(gq[oc], gl8);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float w = p.norm_weight ? __ldg(p.norm_weight + wg * 64 + 8 * oc + e) : 1.f;
-                f[e] *= __fdividef(w, 1.f + ex2(-gl8[e] * kLog2e));
-              }
-            }
-            op[oc] = pack8(f);
-          }
-        }
-      }
-      sync_for_mma();  // the bf16 state copy feeds the next chunk's UMMAs
-      if (*(volatile int32_t*)&m->abort) { ok = false; break; }
+      L_prev = L;
+      tok_prev = tok;
+    }
+    if (ok && write_out && nchunks > 0) {
+      load_gate(L_prev, tok_prev);
+      epilogue(L_prev, tok_prev);
     }
 
     // ---------------------------------------------------------------- end state
@@ -673,6 +765,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (seg.role == kRoleHead) {
         dst = p.ws_state + ((size_t)(seg.slot + 1) * H + h) * unit_state;
       }
+      size_t ld = DV;
+      if (seg.role == kRoleLocalS || seg.role == kRoleLocalM) {  // (S_loc | M) block, row stride dv + dk
+        ld = DV + DK;
+        dst = p.ws_local + ((size_t)seg.slot * H + h) * (size_t)DK * ld + (seg.role == kRoleLocalM ? DV : 0);
+      }
       if (dst) {
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
@@ -682,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int jj = 0; jj < 32; jj += 4)
-            *reinterpret_cast<float4*>(dst + (size_t)row * DV + c0 + jj) =
+            *reinterpret_cast<float4*>(dst + (size_t)row * ld + c0 + jj) =
                 make_float4(__uint_as_float(v[jj]), __uint_as_float(v[jj + 1]), __uint_as_float(v[jj + 2]),
                             __uint_as_float(v[jj + 3]));
         }

@@ -24,6 +24,11 @@ enum SegRole : int32_t {
                       //   end state -> workspace start-state slot of the next segment
   kRoleFromWs = 3,    // split pass 2: start from workspace start-state slot; writes outputs;
                       //   end state -> final_state if last segment of its sequence
+  kRoleLocalS = 4,    // split pass 1 on the tensor-core kernel: start from 0, no outputs;
+                      //   end state -> columns [0, dv) of the slot's (S_loc | M) block
+  kRoleLocalM = 5,    // split pass 1 on the tensor-core kernel: start from I with values taken
+                      //   as zero (so the end state is the segment's transition M), no outputs;
+                      //   end state -> columns [dv, dv + dk) of the slot's (S_loc | M) block
 };
 
 struct Seg {
