@@ -166,6 +166,28 @@ typedef struct kda_decode_args {
 
 kda_status kda_decode_step(const kda_decode_args* args, void* cuda_stream);
 
+/* ------------------------------------------------------------------------------------------
+ * kda_chunk_fwd without a caller-provided workspace.  The paper has no counterpart: this is a
+ * deployment convenience for callers that cannot allocate device memory themselves, e.g. code
+ * running inside a CUDA graph that is being captured, or inside an inference runtime whose
+ * memory pool is fixed at start-up.  Such callers still pass inputs and outputs, but instead of
+ * args->workspace (ignored) the call uses a scratch array that the library holds in static
+ * device memory: KDA_NOALLOC_SCRATCH_BYTES on every GPU that loads the library, kept until the
+ * process exits.
+ *   - A request needing more scratch than that (see kda_chunk_fwd_workspace_size; long
+ *     sequences split across SMs need the most) returns KDA_ERR_WORKSPACE_TOO_SMALL before
+ *     anything is launched.
+ *   - The first call on each device looks up the array's device address with that device
+ *     current; make that first call before any stream capture.  No call allocates memory.
+ *   - All calls share the one array: calls that may overlap on the GPU (different streams,
+ *     concurrent threads) race on it.  Serialise them, or use kda_chunk_fwd with a workspace.
+ *   - The array keeps the last call's contents; each call clears the error word it needs.
+ *   - error_word (may be NULL) receives the device address of the error word for
+ *     kda_read_device_error; it stays valid, and is overwritten by the next call.
+ * ------------------------------------------------------------------------------------------ */
+#define KDA_NOALLOC_SCRATCH_BYTES (32u << 20)
+kda_status kda_chunk_fwd_noalloc(const kda_chunk_args* args, void* cuda_stream, const void** error_word);
+
 /* Synchronise `cuda_stream`, read the device error word (a kda_chunk_fwd workspace or a
  * decode error_word), reset it to zero and return the status it held (KDA_OK if none).
  * Returns KDA_ERR_CUDA if the synchronisation or the copy fails. */

@@ -36,7 +36,8 @@ KDA_FLAG_FORCE_SIMT = 0x2
 KDA_FLAG_TEST_FORCE_TIMEOUT = 0x4
 
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
-            "kda_read_device_error", "kda_status_string")
+            "kda_read_device_error", "kda_status_string", "kda_chunk_fwd_noalloc")
+KDA_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _P = ctypes.c_void_p
 
@@ -95,6 +96,8 @@ def lib():
             L.kda_decode_step.restype = ctypes.c_int
             L.kda_read_device_error.argtypes = [_P, _P]
             L.kda_read_device_error.restype = ctypes.c_int
+            L.kda_chunk_fwd_noalloc.argtypes = [ctypes.POINTER(KdaChunkArgs), _P, ctypes.POINTER(ctypes.c_void_p)]
+            L.kda_chunk_fwd_noalloc.restype = ctypes.c_int
             L.kda_status_string.argtypes = [ctypes.c_int]
             L.kda_status_string.restype = ctypes.c_char_p
             _lib = L
@@ -210,6 +213,33 @@ def kda_chunk_fwd(q, k, v, g, beta, *, gate=None, cu_seqlens=None, initial_state
     if rc != KDA_OK:
         raise KdaError(rc, "kda_chunk_fwd")
     return out, final_state, workspace
+
+
+def kda_chunk_fwd_noalloc(q, k, v, g, beta, *, gate=None, cu_seqlens=None, initial_state=None,
+                          norm_weight=None, output_final_state=True, scale=0.0, eps=1e-6, flags=0,
+                          split_segments=0, out=None, final_state=None, stream=None):
+    """kda_chunk_fwd through the entry point that needs no workspace: for callers that cannot
+    allocate device memory, the library's static scratch array is used (see include/kda.h).
+    Returns (out, final_state, error_word_address)."""
+    _check_cuda(q, k, v, g, beta, gate, initial_state, norm_weight)
+    if isinstance(cu_seqlens, torch.Tensor):
+        cu_seqlens = cu_seqlens.cpu().numpy()
+    if out is None:
+        out = torch.empty(v.shape, dtype=v.dtype, device=v.device)
+    if final_state is None and output_final_state:
+        num_seqs = q.shape[0] if q.dim() == 4 else (1 if cu_seqlens is None else len(cu_seqlens) - 1)
+        final_state = torch.empty((num_seqs, q.shape[-2], q.shape[-1], v.shape[-1]),
+                                  dtype=torch.float32, device=q.device)
+    a, keep = make_chunk_args(q, k, v, g, beta, gate=gate, cu_seqlens=cu_seqlens,
+                              initial_state=initial_state, norm_weight=norm_weight, out=out,
+                              final_state=final_state, scale=scale, eps=eps, flags=flags,
+                              split_segments=split_segments)
+    err = ctypes.c_void_p(0)
+    rc = lib().kda_chunk_fwd_noalloc(ctypes.byref(a), _stream(stream), ctypes.byref(err))
+    del keep
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd_noalloc")
+    return out, final_state, int(err.value or 0)
 
 
 def kda_decode_step(q, k, v, g, beta, state, *, gate=None, state_indices=None, norm_weight=None,
