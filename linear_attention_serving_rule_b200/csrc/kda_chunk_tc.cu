@@ -21,17 +21,19 @@
 // operand Kc_a = k e^{r_a - gamma} over the first 16(a+1) tokens; one M=128 UMMA per a
 // produces A (rows 0-63) and P (rows 64-127) from the stacked operand [k; q] e^{gamma - r_own}.
 //
-// Work split (288 threads): warp 8 is the TMA producer (k and q land interleaved as one
-// 128-row tile, g and v beside them; q/k/g are handed back as soon as the Gram UMMAs have
-// read them, v after the W/U' UMMAs); warps 0-7 are two compute warpgroups.  Warp w owns
-// TMEM lane quarter w % 4 and works on column half w / 4, so every CUDA-core phase (decay
-// prep, Gram read-out, UT inverse, -W/U conversion, state copy, epilogue) runs on 256
-// threads; thread 0 issues the UMMAs.  The gate logits are read straight from global memory
-// by the epilogue.
+// Work split (288 threads): warp 8 is the TMA producer with three groups of tiles: g (with beta,
+// handed back right after the decay scan), k and q (landing interleaved as one 128-row tile;
+// handed back after the UMMAs that read their in-place products) and v (after W/U').  Warps 0-7
+// are two compute warpgroups; warp w owns TMEM lane quarter w % 4.  Decay prep, Gram read-out,
+// UT inverse and the -W / U conversions run on all 256 threads; in the shadow of the Gram UMMAs
+// warpgroup 0 runs the previous chunk's epilogue while warpgroup 1 copies and decays the state.
+// Thread 0 issues the UMMAs.  The gate logits are staged from global memory with cp.async.
 //
 // TMEM (512 columns allocated): [0,128) the fp32 state S (M=128; decayed in place while the
 // Gram UMMAs run, then K^T U accumulated onto it); [128,288) A|P (M=128, N = 16,32,48,64);
-// [288,416) W / O at lane offset 0 and U' -> U at lane offset 16 (two interleaved M=64 tiles).
+// [288,352) W -> O and [352,416) U' -> U: each M=64 product is issued as two N=64 halves, columns
+// 0-63 at lane offset 0 and columns 64-127 at lane offset 16 of the same TMEM columns, so a warp's
+// 32 lanes read 16 rows x 2 column halves and every lane takes part in the read-outs.
 //
 // Every wait is bounded (%globaltimer): on expiry the kernel records KDA_ERR_TIMEOUT, stops
 // issuing work, drains its own in-flight TMA and UMMA operations (bounded again), frees TMEM
@@ -57,7 +59,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr uint32_t OFF_KQ = 0;       // k rows 0-63 | q rows 64-127 (TMA); later e^{gamma} k | e^{gamma} q in place
 constexpr uint32_t OFF_G = 32768;    // g (TMA)
 constexpr uint32_t OFF_V = 49152;    // v (TMA), B operand of U' = T' V
-constexpr uint32_t OFF_KC = 65536;   // Kc_0..Kc_3 (40 KB); then fp32 A and T of the inverse
+constexpr uint32_t OFF_KC = 65536;   // stacked Kc_0..Kc_3 (160 rows, 40 KB); then fp32 A and T of the inverse
 constexpr uint32_t OFF_KL = 106496;  // [k; q] e^{gamma - r_own} (128 rows, 32 KB); then -W; then U
 constexpr uint32_t OFF_KH = 139264;  // e^{gamma_C - gamma} k
 constexpr uint32_t OFF_S = 155648;   // bf16 state, MN-major [dk rows][dv], two 16 KB column blocks
@@ -71,19 +73,19 @@ constexpr int LDT = 68;  // row stride of T (16-byte aligned rows for float4 acc
 
 constexpr uint32_t TM_S = 0, TM_AP = 128, TM_WU = 288;
 
-// Kc_a (16(a+1) rows, two column blocks of 16(a+1) x 128 bytes) inside OFF_KC
-__host__ __device__ constexpr uint32_t kc_off(int a) { return a == 0 ? 0u : a == 1 ? 4096u : a == 2 ? 12288u : 24576u; }
-// column offset of the A|P accumulator of sub-tile a (N = 16, 32, 48, 64)
+// The column operands Kc_0..Kc_3 (16(a+1) rows each) are stacked into one 160-row K-major tile
+// (two 64-column blocks of 160 x 128 bytes); Kc_a starts at row ap_off(a), which is also the
+// TMEM column offset of sub-tile a's block of A|P, so one N=160 UMMA produces all of A|P.
 __host__ __device__ constexpr uint32_t ap_off(int a) { return a == 0 ? 0u : a == 1 ? 16u : a == 2 ? 48u : 96u; }
+constexpr uint32_t KC_ROWS = 160, KC_BLK = KC_ROWS * 128;
 
 struct Misc {
-  uint64_t full_qkg, full_v, empty_qkg, empty_v, mma;
+  uint64_t full_g, full_kq, full_v, empty_g, empty_kq, empty_v, mma;
   uint32_t tmem_base;
   int32_t abort;
   float beta[2][C];  // double-buffered by chunk parity (written by the producer warp)
   float se[4][DK];  // e^{decay over sub-tile m}, per channel
   float ec[DK];     // e^{gamma_C}
-  float ss[2][C];   // epilogue: partial sums of squares of the two column halves
   float y[768];     // inverse scratch
 };
 static_assert(sizeof(Misc) <= 8192, "misc block too large");
@@ -138,14 +140,18 @@ __device__ __forceinline__ uint4& at16(uint8_t* base, uint32_t off) { return *re
 
 // Issue the K loop of one UMMA.  K-major operands step 32 bytes per 16-wide K step and jump to
 // their second 64-column block (blk bytes away) after 4 steps; MN-major ones step 2048 bytes.
+// The descriptors are built once; each K step only adds its byte offset / 16 to the start-address
+// field (bits 0-13), which cannot carry out for shared-memory addresses.
 __device__ __forceinline__ void umma_k_loop(uint32_t d, uint32_t a_addr, uint32_t a_lbo, bool a_kmajor,
                                             uint32_t a_blk, uint32_t b_addr, uint32_t b_lbo, bool b_kmajor,
                                             uint32_t b_blk, int ksteps, uint32_t idesc, bool accumulate) {
+  const uint64_t a0 = smem_desc_sw128(a_addr, a_lbo, 1024);
+  const uint64_t b0 = smem_desc_sw128(b_addr, b_lbo, 1024);
+#pragma unroll
   for (int k = 0; k < ksteps; ++k) {
     const uint32_t ao = a_kmajor ? (uint32_t)(k >> 2) * a_blk + (uint32_t)(k & 3) * 32u : (uint32_t)k * 2048u;
     const uint32_t bo = b_kmajor ? (uint32_t)(k >> 2) * b_blk + (uint32_t)(k & 3) * 32u : (uint32_t)k * 2048u;
-    umma_bf16(d, smem_desc_sw128(a_addr + ao, a_lbo, 1024), smem_desc_sw128(b_addr + bo, b_lbo, 1024), idesc,
-              (accumulate || k > 0) ? 1u : 0u);
+    umma_bf16(d, a0 + (ao >> 4), b0 + (bo >> 4), idesc, (accumulate || k > 0) ? 1u : 0u);
   }
 }
 
@@ -169,8 +175,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool need_v = seg.role != kRoleLocalM;  // the transition pass runs with values = 0
 
   if (tid == 0) {
-    mbar_init(&m->full_qkg, 1); mbar_init(&m->full_v, 1);
-    mbar_init(&m->empty_qkg, 1); mbar_init(&m->empty_v, 1);
+    mbar_init(&m->full_g, 1); mbar_init(&m->full_kq, 1); mbar_init(&m->full_v, 1);
+    mbar_init(&m->empty_g, 1); mbar_init(&m->empty_kq, 1); mbar_init(&m->empty_v, 1);
     mbar_init(&m->mma, 1);
     m->abort = 0;
     fence_mbar_init();
@@ -190,14 +196,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 8) {
     // ===================================================================== TMA producer
     // Lane 0 issues the tile loads; the whole warp first fetches the chunk's beta into the
-    // double buffer m->beta[j & 1] (published by the same mbarrier as the q/k/g tiles).
-    int iq = -1, iv = -1;  // last chunk whose q/k/g and v loads were issued
+    // double buffer m->beta[j & 1], published by the same mbarrier as the g tile.
+    int ig = -1, ikq = -1, iv = -1;  // last chunk whose g, k|q and v loads were issued
     for (int j = 0; j < nchunks; ++j) {
       const int32_t tok = seg.tok0 + j * C;
       const int L = min(C, seg.len - j * C);
       const uint32_t par = (uint32_t)((j & 1) ^ 1);
       int okw = 1;
-      if (lane == 0) okw = wait_bounded(&m->empty_qkg, par, m, drain_limit, p.error_word) ? 1 : 0;
+      if (lane == 0) okw = wait_bounded(&m->empty_g, par, m, drain_limit, p.error_word) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);
       if (!okw) break;
 #pragma unroll
@@ -207,14 +213,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive_expect_tx(&m->full_qkg, 3 * 16384);
+        mbar_arrive_expect_tx(&m->full_g, 16384);
+        for (int hf = 0; hf < 2; ++hf) tma_load_3d(sm + OFF_G + hf * 8192, &maps.g, &m->full_g, hf * 64, h, tok);
+      }
+      ig = j;
+      if (lane == 0) okw = wait_bounded(&m->empty_kq, par, m, drain_limit, p.error_word) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (!okw) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&m->full_kq, 2 * 16384);
         for (int hf = 0; hf < 2; ++hf) {
-          tma_load_3d(sm + OFF_KQ + hf * 16384, &maps.k, &m->full_qkg, hf * 64, h, tok);
-          tma_load_3d(sm + OFF_KQ + hf * 16384 + 8192, &maps.q, &m->full_qkg, hf * 64, h, tok);
-          tma_load_3d(sm + OFF_G + hf * 8192, &maps.g, &m->full_qkg, hf * 64, h, tok);
+          tma_load_3d(sm + OFF_KQ + hf * 16384, &maps.k, &m->full_kq, hf * 64, h, tok);
+          tma_load_3d(sm + OFF_KQ + hf * 16384 + 8192, &maps.q, &m->full_kq, hf * 64, h, tok);
         }
       }
-      iq = j;
+      ikq = j;
       if (!need_v) continue;
       if (lane == 0) okw = wait_bounded(&m->empty_v, par, m, drain_limit, p.error_word) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);
@@ -227,7 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // drain: after an abort, wait (bounded, regardless of the abort) for the loads issued
     if (lane == 0 && *(volatile int32_t*)&m->abort) {
-      if (iq >= 0) wait_bounded(&m->full_qkg, (uint32_t)(iq & 1), m, drain_limit, p.error_word, false);
+      if (ig >= 0) wait_bounded(&m->full_g, (uint32_t)(ig & 1), m, drain_limit, p.error_word, false);
+      if (ikq >= 0) wait_bounded(&m->full_kq, (uint32_t)(ikq & 1), m, drain_limit, p.error_word, false);
       if (iv >= 0) wait_bounded(&m->full_v, (uint32_t)(iv & 1), m, drain_limit, p.error_word, false);
     }
   } else {
@@ -316,52 +330,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       cp_async_commit();
     };
+    // Epilogue of one chunk, run by warpgroup 0 alone: lanes l < 16 of warp q hold columns 0-63
+    // and lanes l + 16 columns 64-127 of O row 16 q + l; the row's sum of squares is combined
+    // across the two lanes with one shuffle.  The gate logits come from the cp.async staging.
     auto epilogue = [&](int L_e, int32_t tok_e) {
-      const int t = 16 * q4 + lane;
-      const bool act = lane < 16 && t < L_e;
+      const int t = 16 * q4 + (lane & 15);
+      const int half = lane >> 4;
+      uint32_t v0[32], v1[32];
+      tmem_ld32(tl + TM_WU, v0);
+      tmem_ld32(tl + TM_WU + 32, v1);
+      tmem_wait_ld();
       float ss = 0.f;
 #pragma unroll
-      for (int hb = 0; hb < 2; ++hb) {
-        uint32_t v[32];
-        tmem_ld32(tl + TM_WU + wg * 64 + 32 * hb, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const float a = __uint_as_float(v[jj]) * p.scale;
-          ss += a * a;
-        }
+      for (int jj = 0; jj < 32; ++jj) {
+        const float a0 = __uint_as_float(v0[jj]), a1 = __uint_as_float(v1[jj]);
+        ss += a0 * a0 + a1 * a1;
       }
-      if (lane < 16) m->ss[wg][t] = ss;
-      cp_async_wait_all();
-      sync_wg();
-      const float rr = (has_gate && lane < 16) ? rsqrtf((m->ss[0][t] + m->ss[1][t]) / (float)DV + p.eps) : 1.f;
+      ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+      if (t >= L_e) return;
+      const float rr = has_gate ? rsqrtf(ss * p.scale * p.scale / (float)DV + p.eps) : 1.f;
       const float sc = p.scale * rr;
       uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ((size_t)(tok_e + t) * H + h) * DV +
-                                           wg * 64);
+                                           half * 64);
 #pragma unroll
-      for (int hb = 0; hb < 2; ++hb) {
-        uint32_t v[32];
-        tmem_ld32(tl + TM_WU + wg * 64 + 32 * hb, v);
-        tmem_wait_ld();
-        if (act) {
+      for (int oc = 0; oc < 8; ++oc) {
+        float f[8];
 #pragma unroll
-          for (int oc = 0; oc < 4; ++oc) {
-            float f[8];
+        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(oc < 4 ? v0[8 * oc + e] : v1[8 * (oc - 4) + e]) * sc;
+        if (has_gate) {
+          float gl8[8];
+          const int c16 = half * 8 + oc;
+          unpack8(at16(sm, OFF_TP + t * 256 + ((c16 ^ (t & 15)) << 4)), gl8);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]) * sc;
-            if (has_gate) {
-              float gl8[8];
-              const int c16 = wg * 8 + 4 * hb + oc;
-              unpack8(at16(sm, OFF_TP + t * 256 + ((c16 ^ (t & 15)) << 4)), gl8);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float w = p.norm_weight ? __ldg(p.norm_weight + wg * 64 + 32 * hb + 8 * oc + e) : 1.f;
-                f[e] *= __fdividef(w, 1.f + ex2(-gl8[e] * kLog2e));
-              }
-            }
-            op[4 * hb + oc] = pack8(f);
+          for (int e = 0; e < 8; ++e) {
+            const float w = p.norm_weight ? __ldg(p.norm_weight + half * 64 + 8 * oc + e) : 1.f;
+            f[e] *= __fdividef(w, 1.f + ex2(-gl8[e] * kLog2e));
           }
         }
+        op[oc] = pack8(f);
       }
     };
 
@@ -373,9 +379,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t par = (uint32_t)(j & 1);
       const float* beta = m->beta[j & 1];
       if (write_out && j > 0) load_gate(L_prev, tok_prev);  // consumed by its epilogue below
-      if (!wg_wait(&m->full_qkg, par)) { ok = false; break; }
+      if (!wg_wait(&m->full_g, par)) { ok = false; break; }
 
-      // ---------------------------------------------------------------- decay prep A: Gram operands
+      // ---------------------------------------------------------------- decay prep: all bf16 operands
       // thread: channels 8o .. 8o+7, tokens t0 .. t0+3 of sub-tile b
       const int qq = tid & 3, o = (tid >> 2) & 15, b = tid >> 6;
       const int t0 = 16 * b + 4 * qq;
@@ -415,31 +421,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (qq == 3) m->se[b][8 * o + e] = ex2(x);  // decay over the whole sub-tile
         }
       }
-      sync_wg();
-      // Per-channel factors, split so that no product of an O(1) value with an underflowed
-      // factor is lost: with se_m = e^{decay over sub-tile m},
-      //   Eb   = e^{r_b}                       = prod_{m<b} se_m
-      //   Rh_a = e^{r_a - r_{b+1}}  (a > b)    = prod_{b<m<a} se_m
-      //   Ehi  = e^{gamma_C - r_{b+1}}         = prod_{m>b} se_m
-      // and per token ix * se_b = e^{r_{b+1} - gamma_t} lies in [e^-80, 1].
-      float Eb[8], Ehi[8], sb[8];
+      // g is consumed (its scan lives in registers): let the producer fetch the next chunk's g,
+      // then wait for this chunk's k and q
+      if (!wg_wait(&m->full_kq, par)) { ok = false; break; }
+      if (tid == 0) mbar_arrive(&m->empty_g);
+      // Per-channel factors, applied so that no O(1) value is multiplied by an underflowed
+      // constant: with se_m = e^{decay over sub-tile m}, Eb = e^{r_b} = prod_{m<b} se_m, and per
+      // token ix = e^{r_b - gamma_t} in [1, e^80]; the chain ix, ix se_b, ix se_b se_{b+1}, ...
+      // gives e^{r_a - gamma_t} for a = b..3, each factor <= 1 after the first.
+      float Eb[8], sb[8];
       {
-        float s1[8], s2[8];  // se_{b+1}, se_{b+2} (1 past the last sub-tile)
+        float s1[8], s2[8], s3[8];  // se_{b+1}, se_{b+2} (1 past the last sub-tile); se_3
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           float se[4];
 #pragma unroll
           for (int mm = 0; mm < 4; ++mm) se[mm] = m->se[mm][8 * o + e];
-          float eb = 1.f, ehi = 1.f;
+          float eb = 1.f;
 #pragma unroll
-          for (int mm = 0; mm < 4; ++mm) {
+          for (int mm = 0; mm < 4; ++mm)
             if (mm < b) eb *= se[mm];
-            if (mm > b) ehi *= se[mm];
-          }
-          Eb[e] = eb; Ehi[e] = ehi;
+          Eb[e] = eb;
           sb[e] = b == 0 ? se[0] : b == 1 ? se[1] : b == 2 ? se[2] : se[3];
           s1[e] = b == 0 ? se[1] : b == 1 ? se[2] : b == 2 ? se[3] : 1.f;
           s2[e] = b == 0 ? se[2] : b == 1 ? se[3] : 1.f;
+          s3[e] = se[3];
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -460,25 +466,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) f[e] = qf[e] * x[e];
           at16(sm, OFF_KL + sw128_oct(64 + t, o, 16384)) = pack8(f);
-          // Kc_a = k e^{r_a - gamma_t}: k ix for a = b, then k ix se_b se_{b+1} ... se_{a-1}
+          // e^{gamma} k and e^{gamma} q, in place over the raw tiles (this thread's own elements)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = kf[e] * x[e] * Eb[e];
+          at16(sm, OFF_KQ + sw128_oct(t, o, 16384)) = pack8(f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = qf[e] * x[e] * Eb[e];
+          at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)) = pack8(f);
+          // Kc_a = k e^{r_a - gamma_t}: k ix for a = b, then k ix se_b se_{b+1} ... se_{a-1};
+          // the last one (a = 3) times se_3 is e^{gamma_C - gamma_t} k, the state-carry operand
 #pragma unroll
           for (int e = 0; e < 8; ++e) f[e] = kf[e] * ix[e];
-          at16(sm, OFF_KC + kc_off(b) + sw128_oct(t, o, 2048u * (b + 1))) = pack8(f);
+          at16(sm, OFF_KC + sw128_oct(ap_off(b) + t, o, KC_BLK)) = pack8(f);
           if (b < 3) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = kf[e] * ix[e] * sb[e];
-            at16(sm, OFF_KC + kc_off(b + 1) + sw128_oct(t, o, 2048u * (b + 2))) = pack8(f);
+            at16(sm, OFF_KC + sw128_oct(ap_off(b + 1) + t, o, KC_BLK)) = pack8(f);
             if (b < 2) {
 #pragma unroll
               for (int e = 0; e < 8; ++e) f[e] *= s1[e];
-              at16(sm, OFF_KC + kc_off(b + 2) + sw128_oct(t, o, 2048u * (b + 3))) = pack8(f);
+              at16(sm, OFF_KC + sw128_oct(ap_off(b + 2) + t, o, KC_BLK)) = pack8(f);
               if (b < 1) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e) f[e] *= s2[e];
-                at16(sm, OFF_KC + kc_off(3) + sw128_oct(t, o, 8192u)) = pack8(f);
+                at16(sm, OFF_KC + sw128_oct(ap_off(3) + t, o, KC_BLK)) = pack8(f);
               }
             }
           }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] *= s3[e];
+          at16(sm, OFF_KH + sw128_oct(t, o, 8192)) = pack8(f);
         }
       }
       if (tid < DK) m->ec[tid] = m->se[0][tid] * m->se[1][tid] * m->se[2][tid] * m->se[3][tid];
@@ -486,48 +503,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------------- UMMA: A | P
       if (tid == 0) {
         tc_fence_after();
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          const uint32_t n = 16u * (a + 1);
-          umma_k_loop(tmem + TM_AP + ap_off(a), sm_u + OFF_KL, 16, true, 16384, sm_u + OFF_KC + kc_off(a), 16, true,
-                      n * 128u, 8, idesc_bf16_f32(128, n, 0, 0), false);
-        }
+        umma_k_loop(tmem + TM_AP, sm_u + OFF_KL, 16, true, 16384, sm_u + OFF_KC, 16, true, KC_BLK, 8,
+                    idesc_bf16_f32(128, KC_ROWS, 0, 0), false);
         umma_commit(&m->mma);
       }
       // ---------------------------------------------------------------- in the shadow of the Gram UMMAs:
-      // (1) decay prep B, in place over the raw tiles: e^{gamma} k over k, e^{gamma} q over q,
-      //     and e^{gamma_C - gamma} k
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int t = t0 + i;
-        float kf[8], qf[8], x[8], f[8];
-        if (t < L) {
-          unpack8(at16(sm, OFF_KQ + sw128_oct(t, o, 16384)), kf);
-          unpack8(at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)), qf);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) { kf[e] = 0.f; qf[e] = 0.f; }
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = ex2(gl[i][e]);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = kf[e] * x[e] * Eb[e];
-        at16(sm, OFF_KQ + sw128_oct(t, o, 16384)) = pack8(f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = qf[e] * x[e] * Eb[e];
-        at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)) = pack8(f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = kf[e] * ex2(-gl[i][e]) * sb[e] * Ehi[e];
-        at16(sm, OFF_KH + sw128_oct(t, o, 8192)) = pack8(f);
-      }
-      // (2) the previous chunk's epilogue (its O is still in TMEM)
-      if (write_out && j > 0) epilogue(L_prev, tok_prev);
-      // (3) bf16 copy of the chunk's start state for the UMMAs, then S <- Diag(e^{gamma_C}) S in place
-      {
+      // warpgroup 0: the previous chunk's epilogue (its O is still in TMEM);
+      // warpgroup 1: bf16 copy of the chunk's start state for the UMMAs, then
+      // S <- Diag(e^{gamma_C}) S in place
+      cp_async_wait_all();
+      sync_wg();  // the staged gate logits are visible to every thread
+      if (wg == 0) {
+        if (write_out && j > 0) epilogue(L_prev, tok_prev);
+      } else {
         const float ec = m->ec[row];
 #pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-          const int c0 = wg * 64 + hb * 32;
+        for (int cb = 0; cb < 4; ++cb) {
+          const int c0 = 32 * cb;
           uint32_t v[32];
           tmem_ld32(tl + TM_S + c0, v);
           tmem_wait_ld();
@@ -617,40 +609,40 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < 16; ++i) Tf[(o + i) * LDT + o + jc] = col[i];
         }
         sync_wg();
+        // each thread: a 2-row x 4-column strip of one 16x16 block (32 threads per block)
 #pragma unroll
         for (int d = 1; d <= 3; ++d) {
-          const int nstrip = (4 - d) * 64;  // (block, row, 4-column strip)
-          const int b = tid >> 6, i = (tid >> 2) & 15, j0 = (tid & 3) * 4, a = b + d;
-          if (tid < nstrip) {  // Y = L_{a, blocks b..a-1} T_{blocks b..a-1, b}
-            const float* lrow = Lf + (16 * a + i) * LDF + 16 * b;
+          const int nthr = (4 - d) * 32;
+          const int b = tid >> 5, i0 = ((tid >> 2) & 7) * 2, j0 = (tid & 3) * 4, a = b + d;
+          if (tid < nthr) {  // Y = L_{a, blocks b..a-1} T_{blocks b..a-1, b}
+            const float* l0 = Lf + (16 * a + i0) * LDF + 16 * b;
             const float* tcol = Tf + 16 * b * LDT + 16 * b + j0;
-            float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+            float4 y0 = make_float4(0.f, 0.f, 0.f, 0.f), y1 = y0;
 #pragma unroll
-            for (int cc = 0; cc < 16 * d; cc += 2) {
-              const float l0 = lrow[cc], l1 = lrow[cc + 1];
-              const float4 t0v = *reinterpret_cast<const float4*>(tcol + cc * LDT);
-              const float4 t1v = *reinterpret_cast<const float4*>(tcol + (cc + 1) * LDT);
-              acc0.x += l0 * t0v.x; acc0.y += l0 * t0v.y; acc0.z += l0 * t0v.z; acc0.w += l0 * t0v.w;
-              acc1.x += l1 * t1v.x; acc1.y += l1 * t1v.y; acc1.z += l1 * t1v.z; acc1.w += l1 * t1v.w;
+            for (int cc = 0; cc < 16 * d; ++cc) {
+              const float la = l0[cc], lb = l0[LDF + cc];
+              const float4 tv = *reinterpret_cast<const float4*>(tcol + cc * LDT);
+              y0.x += la * tv.x; y0.y += la * tv.y; y0.z += la * tv.z; y0.w += la * tv.w;
+              y1.x += lb * tv.x; y1.y += lb * tv.y; y1.z += lb * tv.z; y1.w += lb * tv.w;
             }
-            *reinterpret_cast<float4*>(Y + 4 * tid) =
-                make_float4(acc0.x + acc1.x, acc0.y + acc1.y, acc0.z + acc1.z, acc0.w + acc1.w);
+            *reinterpret_cast<float4*>(Y + (b * 16 + i0) * 16 + j0) = y0;
+            *reinterpret_cast<float4*>(Y + (b * 16 + i0 + 1) * 16 + j0) = y1;
           }
           sync_wg();
-          if (tid < nstrip) {  // T_ab = -T_aa Y  (T_aa is lower triangular with exact zeros above)
-            const float* trow = Tf + (16 * a + i) * LDT + 16 * a;
+          if (tid < nthr) {  // T_ab = -T_aa Y  (T_aa is lower triangular with exact zeros above)
+            const float* t0r = Tf + (16 * a + i0) * LDT + 16 * a;
             const float* ycol = Y + (b * 16) * 16 + j0;
-            float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+            float4 u0 = make_float4(0.f, 0.f, 0.f, 0.f), u1 = u0;
 #pragma unroll
-            for (int kk = 0; kk < 16; kk += 2) {
-              const float u0 = trow[kk], u1 = trow[kk + 1];
-              const float4 y0 = *reinterpret_cast<const float4*>(ycol + kk * 16);
-              const float4 y1 = *reinterpret_cast<const float4*>(ycol + (kk + 1) * 16);
-              acc0.x += u0 * y0.x; acc0.y += u0 * y0.y; acc0.z += u0 * y0.z; acc0.w += u0 * y0.w;
-              acc1.x += u1 * y1.x; acc1.y += u1 * y1.y; acc1.z += u1 * y1.z; acc1.w += u1 * y1.w;
+            for (int kk = 0; kk < 16; ++kk) {
+              const float ta = t0r[kk], tb = t0r[LDT + kk];
+              const float4 yv = *reinterpret_cast<const float4*>(ycol + kk * 16);
+              u0.x += ta * yv.x; u0.y += ta * yv.y; u0.z += ta * yv.z; u0.w += ta * yv.w;
+              u1.x += tb * yv.x; u1.y += tb * yv.y; u1.z += tb * yv.z; u1.w += tb * yv.w;
             }
-            *reinterpret_cast<float4*>(Tf + (16 * a + i) * LDT + 16 * b + j0) =
-                make_float4(-(acc0.x + acc1.x), -(acc0.y + acc1.y), -(acc0.z + acc1.z), -(acc0.w + acc1.w));
+            *reinterpret_cast<float4*>(Tf + (16 * a + i0) * LDT + 16 * b + j0) = make_float4(-u0.x, -u0.y, -u0.z, -u0.w);
+            *reinterpret_cast<float4*>(Tf + (16 * a + i0 + 1) * LDT + 16 * b + j0) =
+                make_float4(-u1.x, -u1.y, -u1.z, -u1.w);
           }
           sync_wg();
         }
@@ -677,65 +669,71 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*(volatile int32_t*)&m->abort) { ok = false; break; }
       if (tid == 0) {
         tc_fence_after();
-        const uint32_t id = idesc_bf16_f32(64, 128, 0, 1);
-        umma_k_loop(tmem + TM_WU, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ, 16384, false, 0, 4, id, false);
-        if (need_v)
-          umma_k_loop(tmem + TM_WU + (16u << 16), sm_u + OFF_TP, 16, true, 0, sm_u + OFF_V, 8192, false, 0, 4, id,
+        // columns 0-63 at lane offset 0, 64-127 at lane offset 16: W in [288,352), U' in [352,416)
+        // with values: one N=128 UMMA per half, whose B operand is [e^g k block | v block] -- two
+        // MN atoms (OFF_V - OFF_KQ) and (OFF_V + 8192 - OFF_KQ - 16384) bytes apart -- so D gets
+        // W in [288,352) and U' in [352,416)
+        const uint32_t hi = 16u << 16;
+        if (need_v) {
+          const uint32_t id = idesc_bf16_f32(64, 128, 0, 1);
+          umma_k_loop(tmem + TM_WU, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ, OFF_V - OFF_KQ, false, 0, 4, id, false);
+          umma_k_loop(tmem + TM_WU + hi, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ + 16384, OFF_V + 8192 - OFF_KQ - 16384,
+                      false, 0, 4, id, false);
+        } else {
+          const uint32_t id = idesc_bf16_f32(64, 64, 0, 1);
+          umma_k_loop(tmem + TM_WU, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ, 16384, false, 0, 4, id, false);
+          umma_k_loop(tmem + TM_WU + hi, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ + 16384, 16384, false, 0, 4, id,
                       false);
+        }
       }
       if (!mma_commit_wait()) { ok = false; break; }
       if (tid == 0 && need_v) mbar_arrive(&m->empty_v);
 
-      // ---------------------------------------------------------------- -W -> bf16 (rows of the lane-0 tile)
+      // ---------------------------------------------------------------- -W -> bf16
+      // lane l < 16: row 16 q + l, columns 32 wg ..; lane l + 16: the same row, columns 64 + 32 wg ..
       {
-        const int t = 16 * q4 + lane;  // valid for lane < 16
+        const int t = 16 * q4 + (lane & 15);
+        const int c0 = (lane >> 4) * 64 + wg * 32;
+        uint32_t v[32];
+        tmem_ld32(tl + TM_WU + 32 * wg, v);
+        tmem_wait_ld();
 #pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-          const int c0 = wg * 64 + hb * 32;
-          uint32_t v[32];
-          tmem_ld32(tl + TM_WU + c0, v);
-          tmem_wait_ld();
-          if (lane < 16) {
+        for (int oc = 0; oc < 4; ++oc) {
+          float f[8];
 #pragma unroll
-            for (int oc = 0; oc < 4; ++oc) {
-              float f[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) f[e] = -__uint_as_float(v[8 * oc + e]);
-              at16(sm, OFF_KL + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
-            }
-          }
+          for (int e = 0; e < 8; ++e) f[e] = -__uint_as_float(v[8 * oc + e]);
+          at16(sm, OFF_KL + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
         }
       }
       sync_for_mma();
       // ---------------------------------------------------------------- UMMA: U = U' - W S0 ; O = Qt S0
       if (tid == 0) {
         tc_fence_after();
-        const uint32_t id = idesc_bf16_f32(64, 128, 0, 1);
-        umma_k_loop(tmem + TM_WU + (16u << 16), sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S, 16384, false, 0, 8, id,
-                    need_v);
+        const uint32_t id = idesc_bf16_f32(64, 64, 0, 1);
+        const uint32_t hi = 16u << 16;
+        umma_k_loop(tmem + TM_WU + 64, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S, 16384, false, 0, 8, id, need_v);
+        umma_k_loop(tmem + TM_WU + 64 + hi, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S + 16384, 16384, false, 0, 8,
+                    id, need_v);
         umma_k_loop(tmem + TM_WU, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S, 16384, false, 0, 8, id, false);
+        umma_k_loop(tmem + TM_WU + hi, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S + 16384, 16384, false, 0, 8,
+                    id, false);
       }
       if (!mma_commit_wait()) { ok = false; break; }
-      if (tid == 0) mbar_arrive(&m->empty_qkg);  // k, q, g and their in-place products consumed
+      if (tid == 0) mbar_arrive(&m->empty_kq);  // k, q and their in-place products consumed
 
-      // ---------------------------------------------------------------- U -> bf16 (rows of the lane-16 tile)
+      // ---------------------------------------------------------------- U -> bf16 (same lane split as -W)
       {
-        const int t = 16 * q4 + lane - 16;  // valid for lane >= 16
+        const int t = 16 * q4 + (lane & 15);
+        const int c0 = (lane >> 4) * 64 + wg * 32;
+        uint32_t v[32];
+        tmem_ld32(tl + TM_WU + 64 + 32 * wg, v);
+        tmem_wait_ld();
 #pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-          const int c0 = wg * 64 + hb * 32;
-          uint32_t v[32];
-          tmem_ld32(tl + TM_WU + c0, v);
-          tmem_wait_ld();
-          if (lane >= 16) {
+        for (int oc = 0; oc < 4; ++oc) {
+          float f[8];
 #pragma unroll
-            for (int oc = 0; oc < 4; ++oc) {
-              float f[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
-              at16(sm, OFF_KL + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
-            }
-          }
+          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
+          at16(sm, OFF_KL + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
         }
       }
       sync_for_mma();
@@ -743,7 +741,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid == 0) {
         tc_fence_after();
         umma_k_loop(tmem + TM_WU, sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL, 8192, false, 0, 4,
-                    idesc_bf16_f32(64, 128, 0, 1), true);
+                    idesc_bf16_f32(64, 64, 0, 1), true);
+        umma_k_loop(tmem + TM_WU + (16u << 16), sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL + 8192, 8192, false, 0, 4,
+                    idesc_bf16_f32(64, 64, 0, 1), true);
         umma_k_loop(tmem + TM_S, sm_u + OFF_KH, 8192, false, 0, sm_u + OFF_KL, 8192, false, 0, 4,
                     idesc_bf16_f32(128, 128, 1, 1), true);
       }
@@ -754,7 +754,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && write_out && nchunks > 0) {
       load_gate(L_prev, tok_prev);
-      epilogue(L_prev, tok_prev);
+      cp_async_wait_all();
+      sync_wg();
+      if (wg == 0) epilogue(L_prev, tok_prev);
     }
 
     // ---------------------------------------------------------------- end state
