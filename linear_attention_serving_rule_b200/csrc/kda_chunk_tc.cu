@@ -26,7 +26,8 @@
 // handed back after the UMMAs that read their in-place products) and v (after W/U').  Warps 0-7
 // are two compute warpgroups; warp w owns TMEM lane quarter w % 4.  Decay prep, Gram read-out,
 // UT inverse and the -W / U conversions run on all 256 threads; in the shadow of the Gram UMMAs
-// warpgroup 0 runs the previous chunk's epilogue while warpgroup 1 copies and decays the state.
+// both warpgroups run the previous chunk's epilogue, and while warps 0-1 invert the diagonal
+// blocks of the UT transform, warps 2-7 copy and decay the state.
 // Thread 0 issues the UMMAs.  The gate logits are staged from global memory with cp.async.
 //
 // TMEM (512 columns allocated): [0,128) the fp32 state S (M=128; decayed in place while the
@@ -87,6 +88,8 @@ struct Misc {
   float se[4][DK];  // e^{decay over sub-tile m}, per channel
   float ec[DK];     // e^{gamma_C}
   float y[768];     // inverse scratch
+  float nw[DV];     // RMSNorm weight (1 without one)
+  float ssq[2][C];  // epilogue: per-row sums of squares of the two column halves
 };
 static_assert(sizeof(Misc) <= 8192, "misc block too large");
 
@@ -188,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 8 && lane == 0) {
     prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.g); prefetch_tmap(&maps.v);
   }
+  if (tid < DV) m->nw[tid] = p.norm_weight ? p.norm_weight[tid] : 1.f;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -330,45 +334,70 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       cp_async_commit();
     };
-    // Epilogue of one chunk, run by warpgroup 0 alone: lanes l < 16 of warp q hold columns 0-63
-    // and lanes l + 16 columns 64-127 of O row 16 q + l; the row's sum of squares is combined
-    // across the two lanes with one shuffle.  The gate logits come from the cp.async staging.
+    // Epilogue of one chunk, run by both warpgroups: lanes l < 16 of warp (q, wg) hold columns
+    // 32 wg .. 32 wg + 31 and lanes l + 16 columns 64 + 32 wg .. of O row 16 q + l; a row's sum of
+    // squares is combined across the two lanes with a shuffle and across the warpgroups through
+    // shared memory.  The gate logits come from the cp.async staging.
     auto epilogue = [&](int L_e, int32_t tok_e) {
       const int t = 16 * q4 + (lane & 15);
-      const int half = lane >> 4;
-      uint32_t v0[32], v1[32];
-      tmem_ld32(tl + TM_WU, v0);
-      tmem_ld32(tl + TM_WU + 32, v1);
+      const int c0 = 64 * (lane >> 4) + 32 * wg;
+      uint32_t v[32];
+      tmem_ld32(tl + TM_WU + 32 * wg, v);
       tmem_wait_ld();
       float ss = 0.f;
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) {
-        const float a0 = __uint_as_float(v0[jj]), a1 = __uint_as_float(v1[jj]);
-        ss += a0 * a0 + a1 * a1;
+        const float a0 = __uint_as_float(v[jj]);
+        ss += a0 * a0;
       }
       ss += __shfl_xor_sync(0xffffffffu, ss, 16);
+      if (lane < 16) m->ssq[wg][t] = ss;
+      sync_wg();
+      ss += m->ssq[wg ^ 1][t];
       if (t >= L_e) return;
       const float rr = has_gate ? rsqrtf(ss * p.scale * p.scale / (float)DV + p.eps) : 1.f;
       const float sc = p.scale * rr;
-      uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ((size_t)(tok_e + t) * H + h) * DV +
-                                           half * 64);
+      uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ((size_t)(tok_e + t) * H + h) * DV + c0);
 #pragma unroll
-      for (int oc = 0; oc < 8; ++oc) {
+      for (int oc = 0; oc < 4; ++oc) {
         float f[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(oc < 4 ? v0[8 * oc + e] : v1[8 * (oc - 4) + e]) * sc;
+        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]) * sc;
         if (has_gate) {
           float gl8[8];
-          const int c16 = half * 8 + oc;
+          const int c16 = (c0 >> 3) + oc;
           unpack8(at16(sm, OFF_TP + t * 256 + ((c16 ^ (t & 15)) << 4)), gl8);
+          const float4 w0 = *reinterpret_cast<const float4*>(&m->nw[c0 + 8 * oc]);
+          const float4 w1 = *reinterpret_cast<const float4*>(&m->nw[c0 + 8 * oc + 4]);
+          const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float w = p.norm_weight ? __ldg(p.norm_weight + half * 64 + 8 * oc + e) : 1.f;
-            f[e] *= __fdividef(w, 1.f + ex2(-gl8[e] * kLog2e));
-          }
+          for (int e = 0; e < 8; ++e) f[e] *= __fdividef(w[e], 1.f + ex2(-gl8[e] * kLog2e));
         }
         op[oc] = pack8(f);
       }
+    };
+    // bf16 copy of the state S for the UMMAs, then S <- Diag(e^{gamma_C}) S in TMEM, over the
+    // 32-column blocks [cb0, cb1) of this warp's 32 rows
+    auto state_copy = [&](int cb0, int cb1) {
+      const float ec = m->ec[row];
+#pragma unroll 1
+      for (int cb = cb0; cb < cb1; ++cb) {
+        const int c0 = 32 * cb;
+        uint32_t v[32];
+        tmem_ld32(tl + TM_S + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int oc = 0; oc < 4; ++oc) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
+          at16(sm, OFF_S + sw128_oct(row, (c0 >> 3) + oc, 16384)) = pack8(f);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) v[jj] = __float_as_uint(__uint_as_float(v[jj]) * ec);
+        tmem_st32(tl + TM_S + c0, v);
+      }
+      tmem_wait_st();
     };
 
     int L_prev = 0;
@@ -508,34 +537,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(&m->mma);
       }
       // ---------------------------------------------------------------- in the shadow of the Gram UMMAs:
-      // warpgroup 0: the previous chunk's epilogue (its O is still in TMEM);
-      // warpgroup 1: bf16 copy of the chunk's start state for the UMMAs, then
-      // S <- Diag(e^{gamma_C}) S in place
+      // the previous chunk's epilogue (its O is still in TMEM)
       cp_async_wait_all();
       sync_wg();  // the staged gate logits are visible to every thread
-      if (wg == 0) {
-        if (write_out && j > 0) epilogue(L_prev, tok_prev);
-      } else {
-        const float ec = m->ec[row];
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-          const int c0 = 32 * cb;
-          uint32_t v[32];
-          tmem_ld32(tl + TM_S + c0, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int oc = 0; oc < 4; ++oc) {
-            float f[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
-            at16(sm, OFF_S + sw128_oct(row, (c0 >> 3) + oc, 16384)) = pack8(f);
-          }
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) v[jj] = __float_as_uint(__uint_as_float(v[jj]) * ec);
-          tmem_st32(tl + TM_S + c0, v);
-        }
-        tmem_wait_st();
-      }
+      if (write_out && j > 0) epilogue(L_prev, tok_prev);
       {
         const bool r = wg_wait(&m->mma, mph & 1u);
         ++mph;
@@ -607,42 +612,48 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
           for (int i = 0; i < 16; ++i) Tf[(o + i) * LDT + o + jc] = col[i];
+        } else {
+          // meanwhile warps 2-7 copy and decay the state: warps 4 and 5 own TMEM lane quarters 0
+          // and 1 alone, warps 2|6 and 3|7 share quarters 2 and 3
+          if (q4 < 2) state_copy(0, 4);
+          else state_copy(warp < 4 ? 0 : 2, warp < 4 ? 2 : 4);
         }
         sync_wg();
-        // each thread: a 2-row x 4-column strip of one 16x16 block (32 threads per block)
+        // each thread: a 1-row x 4-column strip of one 16x16 block (64 threads per block)
 #pragma unroll
         for (int d = 1; d <= 3; ++d) {
-          const int nthr = (4 - d) * 32;
-          const int b = tid >> 5, i0 = ((tid >> 2) & 7) * 2, j0 = (tid & 3) * 4, a = b + d;
-          if (tid < nthr) {  // Y = L_{a, blocks b..a-1} T_{blocks b..a-1, b}
-            const float* l0 = Lf + (16 * a + i0) * LDF + 16 * b;
+          const int nstrip = (4 - d) * 64;
+          const int b = tid >> 6, i = (tid >> 2) & 15, j0 = (tid & 3) * 4, a = b + d;
+          if (tid < nstrip) {  // Y = L_{a, blocks b..a-1} T_{blocks b..a-1, b}
+            const float* lrow = Lf + (16 * a + i) * LDF + 16 * b;
             const float* tcol = Tf + 16 * b * LDT + 16 * b + j0;
-            float4 y0 = make_float4(0.f, 0.f, 0.f, 0.f), y1 = y0;
+            float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
 #pragma unroll
-            for (int cc = 0; cc < 16 * d; ++cc) {
-              const float la = l0[cc], lb = l0[LDF + cc];
-              const float4 tv = *reinterpret_cast<const float4*>(tcol + cc * LDT);
-              y0.x += la * tv.x; y0.y += la * tv.y; y0.z += la * tv.z; y0.w += la * tv.w;
-              y1.x += lb * tv.x; y1.y += lb * tv.y; y1.z += lb * tv.z; y1.w += lb * tv.w;
+            for (int cc = 0; cc < 16 * d; cc += 2) {
+              const float l0 = lrow[cc], l1 = lrow[cc + 1];
+              const float4 t0v = *reinterpret_cast<const float4*>(tcol + cc * LDT);
+              const float4 t1v = *reinterpret_cast<const float4*>(tcol + (cc + 1) * LDT);
+              acc0.x += l0 * t0v.x; acc0.y += l0 * t0v.y; acc0.z += l0 * t0v.z; acc0.w += l0 * t0v.w;
+              acc1.x += l1 * t1v.x; acc1.y += l1 * t1v.y; acc1.z += l1 * t1v.z; acc1.w += l1 * t1v.w;
             }
-            *reinterpret_cast<float4*>(Y + (b * 16 + i0) * 16 + j0) = y0;
-            *reinterpret_cast<float4*>(Y + (b * 16 + i0 + 1) * 16 + j0) = y1;
+            *reinterpret_cast<float4*>(Y + 4 * tid) =
+                make_float4(acc0.x + acc1.x, acc0.y + acc1.y, acc0.z + acc1.z, acc0.w + acc1.w);
           }
           sync_wg();
-          if (tid < nthr) {  // T_ab = -T_aa Y  (T_aa is lower triangular with exact zeros above)
-            const float* t0r = Tf + (16 * a + i0) * LDT + 16 * a;
+          if (tid < nstrip) {  // T_ab = -T_aa Y  (T_aa is lower triangular with exact zeros above)
+            const float* trow = Tf + (16 * a + i) * LDT + 16 * a;
             const float* ycol = Y + (b * 16) * 16 + j0;
-            float4 u0 = make_float4(0.f, 0.f, 0.f, 0.f), u1 = u0;
+            float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
 #pragma unroll
-            for (int kk = 0; kk < 16; ++kk) {
-              const float ta = t0r[kk], tb = t0r[LDT + kk];
-              const float4 yv = *reinterpret_cast<const float4*>(ycol + kk * 16);
-              u0.x += ta * yv.x; u0.y += ta * yv.y; u0.z += ta * yv.z; u0.w += ta * yv.w;
-              u1.x += tb * yv.x; u1.y += tb * yv.y; u1.z += tb * yv.z; u1.w += tb * yv.w;
+            for (int kk = 0; kk < 16; kk += 2) {
+              const float u0 = trow[kk], u1 = trow[kk + 1];
+              const float4 y0 = *reinterpret_cast<const float4*>(ycol + kk * 16);
+              const float4 y1 = *reinterpret_cast<const float4*>(ycol + (kk + 1) * 16);
+              acc0.x += u0 * y0.x; acc0.y += u0 * y0.y; acc0.z += u0 * y0.z; acc0.w += u0 * y0.w;
+              acc1.x += u1 * y1.x; acc1.y += u1 * y1.y; acc1.z += u1 * y1.z; acc1.w += u1 * y1.w;
             }
-            *reinterpret_cast<float4*>(Tf + (16 * a + i0) * LDT + 16 * b + j0) = make_float4(-u0.x, -u0.y, -u0.z, -u0.w);
-            *reinterpret_cast<float4*>(Tf + (16 * a + i0 + 1) * LDT + 16 * b + j0) =
-                make_float4(-u1.x, -u1.y, -u1.z, -u1.w);
+            *reinterpret_cast<float4*>(Tf + (16 * a + i) * LDT + 16 * b + j0) =
+                make_float4(-(acc0.x + acc1.x), -(acc0.y + acc1.y), -(acc0.z + acc1.z), -(acc0.w + acc1.w));
           }
           sync_wg();
         }
@@ -756,7 +767,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       load_gate(L_prev, tok_prev);
       cp_async_wait_all();
       sync_wg();
-      if (wg == 0) epilogue(L_prev, tok_prev);
+      epilogue(L_prev, tok_prev);
     }
 
     // ---------------------------------------------------------------- end state
