@@ -68,9 +68,11 @@ constexpr uint32_t OFF_TP = 188416;  // T' = T Diag(beta), bf16 [64][64]
 constexpr uint32_t OFF_P = 196608;   // P (causally masked), bf16 [64][64]
 constexpr uint32_t OFF_MISC = 204800;
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 8192 + 1024;
-constexpr uint32_t OFF_TF = OFF_KC + 16640;  // fp32 T [64][68], after fp32 A [64][65]
-constexpr int LDF = 65;  // row stride of A (scalar column writes, conflict-free)
-constexpr int LDT = 68;  // row stride of T (16-byte aligned rows for float4 access)
+// fp32 L = Diag(beta) A [64][68], then fp32 T [64][68]: a row stride of 4 mod 32 words keeps the
+// mma.sync A-fragment loads (8 rows x 4 columns per warp) free of bank conflicts
+constexpr int LDF = 68;
+constexpr int LDT = 68;
+constexpr uint32_t OFF_TF = OFF_KC + 64 * LDF * 4;
 
 constexpr uint32_t TM_S = 0, TM_AP = 128, TM_WU = 288;
 
@@ -87,7 +89,6 @@ struct Misc {
   float beta[2][C];  // double-buffered by chunk parity (written by the producer warp)
   float se[4][DK];  // e^{decay over sub-tile m}, per channel
   float ec[DK];     // e^{gamma_C}
-  float y[768];     // inverse scratch
   float nw[DV];     // RMSNorm weight (1 without one)
   float ssq[2][C];  // epilogue: per-row sums of squares of the two column halves
 };
@@ -140,6 +141,39 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 __device__ __forceinline__ uint4& at16(uint8_t* base, uint32_t off) { return *reinterpret_cast<uint4*>(base + off); }
+
+// Warp-level m16n8k8 tf32 MMA (fp32 accumulate).  Fragments, with g = lane / 4, t = lane % 4:
+// A (16x8): (g, t), (g+8, t), (g, t+4), (g+8, t+4); B (8x8): (t, g), (t+4, g);
+// C (16x8): (g, 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1).
+__device__ __forceinline__ uint32_t tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// fp32-accurate product from three tf32 MMAs: with x = x_hi + x_lo (both tf32), a b ~ a_hi b_hi
+// (into dm) + a_hi b_lo + a_lo b_hi (into dc); the dropped a_lo b_lo is below fp32 rounding.
+__device__ __forceinline__ void mma_3xtf32(float (&dm)[4], float (&dc)[4], const float (&a)[4], const float (&b)[2]) {
+  uint32_t ah[4], al[4], bh[2], bl[2];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    ah[i] = tf32_rna(a[i]);
+    al[i] = tf32_rna(a[i] - __uint_as_float(ah[i]));
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    bh[i] = tf32_rna(b[i]);
+    bl[i] = tf32_rna(b[i] - __uint_as_float(bh[i]));
+  }
+  mma_tf32(dm, ah, bh);
+  mma_tf32(dc, ah, bl);
+  mma_tf32(dc, al, bh);
+}
 
 // Issue the K loop of one UMMA.  K-major operands step 32 bytes per 16-wide K step and jump to
 // their second 64-column block (blk bytes away) after 4 steps; MN-major ones step 2048 bytes.
@@ -595,7 +629,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         const float* Lf = reinterpret_cast<const float*>(sm + OFF_KC);
         float* Tf = reinterpret_cast<float*>(sm + OFF_TF);
-        float* Y = m->y;
         if (tid < 64) {
           const int a = tid >> 4, jc = tid & 15, o = 16 * a;
           float col[16];
@@ -619,43 +652,56 @@ __global__ void __launch_bounds__(kThreads, 1)
           else state_copy(warp < 4 ? 0 : 2, warp < 4 ? 2 : 4);
         }
         sync_wg();
-        // each thread: a 1-row x 4-column strip of one 16x16 block (64 threads per block)
+        // Off-diagonal blocks level by level (block distance d), one 16x8 strip per warp: warp
+        // w < 2 (4 - d) takes a = b + d with b = w / 2 and columns 16 b + 8 (w % 2) .. +7:
+        //   Y = sum_{c=b}^{a-1} L_ac T_cb,   T_ab = -T_aa Y,
+        // as m16n8k8 3xTF32 MMAs.  Y never leaves the warp: its C fragment becomes the B fragment
+        // of the second product by shuffles.  A level reads only blocks of earlier levels.
+        {
+          const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
-        for (int d = 1; d <= 3; ++d) {
-          const int nstrip = (4 - d) * 64;
-          const int b = tid >> 6, i = (tid >> 2) & 15, j0 = (tid & 3) * 4, a = b + d;
-          if (tid < nstrip) {  // Y = L_{a, blocks b..a-1} T_{blocks b..a-1, b}
-            const float* lrow = Lf + (16 * a + i) * LDF + 16 * b;
-            const float* tcol = Tf + 16 * b * LDT + 16 * b + j0;
-            float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
+          for (int d = 1; d <= 3; ++d) {
+            if (warp < 2 * (4 - d)) {
+              const int b = warp >> 1, n0 = 8 * (warp & 1), a = b + d;
+              float ym[4] = {0.f, 0.f, 0.f, 0.f}, yc[4] = {0.f, 0.f, 0.f, 0.f};
+              const float* la = Lf + (16 * a + g) * LDF + t4;
+              const float* tb = Tf + t4 * LDT + 16 * b + n0 + g;
 #pragma unroll
-            for (int cc = 0; cc < 16 * d; cc += 2) {
-              const float l0 = lrow[cc], l1 = lrow[cc + 1];
-              const float4 t0v = *reinterpret_cast<const float4*>(tcol + cc * LDT);
-              const float4 t1v = *reinterpret_cast<const float4*>(tcol + (cc + 1) * LDT);
-              acc0.x += l0 * t0v.x; acc0.y += l0 * t0v.y; acc0.z += l0 * t0v.z; acc0.w += l0 * t0v.w;
-              acc1.x += l1 * t1v.x; acc1.y += l1 * t1v.y; acc1.z += l1 * t1v.z; acc1.w += l1 * t1v.w;
+              for (int ks = 0; ks < 2 * d; ++ks) {
+                const int kk = 16 * b + 8 * ks;
+                const float af[4] = {la[kk], la[8 * LDF + kk], la[kk + 4], la[8 * LDF + kk + 4]};
+                const float bf[2] = {tb[kk * LDT], tb[(kk + 4) * LDT]};
+                mma_3xtf32(ym, yc, af, bf);
+              }
+              float y[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) y[i] = ym[i] + yc[i];
+              // Y[r][n] sits in lane 4 (r % 8) + n / 2, register 2 (r / 8) + n % 2; this lane needs
+              // Y[t][g], Y[t+4][g] (first K step) and Y[8+t][g], Y[12+t][g] (second)
+              const int s0 = 4 * t4 + (g >> 1), s1 = s0 + 16;
+              const bool odd = (g & 1) != 0;
+              float yb[4];
+              {
+                const float u0 = __shfl_sync(0xffffffffu, y[0], s0), v0 = __shfl_sync(0xffffffffu, y[1], s0);
+                const float u1 = __shfl_sync(0xffffffffu, y[0], s1), v1 = __shfl_sync(0xffffffffu, y[1], s1);
+                const float u2 = __shfl_sync(0xffffffffu, y[2], s0), v2 = __shfl_sync(0xffffffffu, y[3], s0);
+                const float u3 = __shfl_sync(0xffffffffu, y[2], s1), v3 = __shfl_sync(0xffffffffu, y[3], s1);
+                yb[0] = odd ? v0 : u0; yb[1] = odd ? v1 : u1; yb[2] = odd ? v2 : u2; yb[3] = odd ? v3 : u3;
+              }
+              float om[4] = {0.f, 0.f, 0.f, 0.f}, oc[4] = {0.f, 0.f, 0.f, 0.f};
+              const float* ta = Tf + (16 * a + g) * LDT + 16 * a + t4;
+#pragma unroll
+              for (int ks = 0; ks < 2; ++ks) {
+                const float af[4] = {-ta[8 * ks], -ta[8 * LDT + 8 * ks], -ta[8 * ks + 4], -ta[8 * LDT + 8 * ks + 4]};
+                const float bf[2] = {yb[2 * ks], yb[2 * ks + 1]};
+                mma_3xtf32(om, oc, af, bf);
+              }
+              float* to = Tf + (16 * a + g) * LDT + 16 * b + n0 + 2 * t4;
+              *reinterpret_cast<float2*>(to) = make_float2(om[0] + oc[0], om[1] + oc[1]);
+              *reinterpret_cast<float2*>(to + 8 * LDT) = make_float2(om[2] + oc[2], om[3] + oc[3]);
             }
-            *reinterpret_cast<float4*>(Y + 4 * tid) =
-                make_float4(acc0.x + acc1.x, acc0.y + acc1.y, acc0.z + acc1.z, acc0.w + acc1.w);
+            sync_wg();
           }
-          sync_wg();
-          if (tid < nstrip) {  // T_ab = -T_aa Y  (T_aa is lower triangular with exact zeros above)
-            const float* trow = Tf + (16 * a + i) * LDT + 16 * a;
-            const float* ycol = Y + (b * 16) * 16 + j0;
-            float4 acc0 = make_float4(0.f, 0.f, 0.f, 0.f), acc1 = acc0;
-#pragma unroll
-            for (int kk = 0; kk < 16; kk += 2) {
-              const float u0 = trow[kk], u1 = trow[kk + 1];
-              const float4 y0 = *reinterpret_cast<const float4*>(ycol + kk * 16);
-              const float4 y1 = *reinterpret_cast<const float4*>(ycol + (kk + 1) * 16);
-              acc0.x += u0 * y0.x; acc0.y += u0 * y0.y; acc0.z += u0 * y0.z; acc0.w += u0 * y0.w;
-              acc1.x += u1 * y1.x; acc1.y += u1 * y1.y; acc1.z += u1 * y1.z; acc1.w += u1 * y1.w;
-            }
-            *reinterpret_cast<float4*>(Tf + (16 * a + i) * LDT + 16 * b + j0) =
-                make_float4(-(acc0.x + acc1.x), -(acc0.y + acc1.y), -(acc0.z + acc1.z), -(acc0.w + acc1.w));
-          }
-          sync_wg();
         }
 #pragma unroll
         for (int it = 0; it < 2; ++it) {
