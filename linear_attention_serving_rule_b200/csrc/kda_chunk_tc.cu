@@ -157,8 +157,9 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 // fp32-accurate product from three tf32 MMAs: with x = x_hi + x_lo (both tf32), a b ~ a_hi b_hi
-// (into dm) + a_hi b_lo + a_lo b_hi (into dc); the dropped a_lo b_lo is below fp32 rounding.
-__device__ __forceinline__ void mma_3xtf32(float (&dm)[4], float (&dc)[4], const float (&a)[4], const float (&b)[2]) {
+// + a_hi b_lo + a_lo b_hi, each term into its own accumulator d[0..2] (three independent MMA
+// chains); the dropped a_lo b_lo is below fp32 rounding.
+__device__ __forceinline__ void mma_3xtf32(float (&d)[3][4], const float (&a)[4], const float (&b)[2]) {
   uint32_t ah[4], al[4], bh[2], bl[2];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -170,9 +171,9 @@ __device__ __forceinline__ void mma_3xtf32(float (&dm)[4], float (&dc)[4], const
     bh[i] = tf32_rna(b[i]);
     bl[i] = tf32_rna(b[i] - __uint_as_float(bh[i]));
   }
-  mma_tf32(dm, ah, bh);
-  mma_tf32(dc, ah, bl);
-  mma_tf32(dc, al, bh);
+  mma_tf32(d[0], ah, bh);
+  mma_tf32(d[1], ah, bl);
+  mma_tf32(d[2], al, bh);
 }
 
 // Issue the K loop of one UMMA.  K-major operands step 32 bytes per 16-wide K step and jump to
@@ -194,8 +195,10 @@ __device__ __forceinline__ void umma_k_loop(uint32_t d, uint32_t a_addr, uint32_
 
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ Plan plan, const __grid_constant__ TcMaps maps, const ChunkParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte aligned base (swizzle atoms), offset by pointer arithmetic on the __shared__ array so
+  // that every access through sm stays a shared-memory access
+  uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   Misc* m = reinterpret_cast<Misc*>(sm + OFF_MISC);
   const uint32_t sm_u = smem_u32(sm);
 
@@ -663,7 +666,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int d = 1; d <= 3; ++d) {
             if (warp < 2 * (4 - d)) {
               const int b = warp >> 1, n0 = 8 * (warp & 1), a = b + d;
-              float ym[4] = {0.f, 0.f, 0.f, 0.f}, yc[4] = {0.f, 0.f, 0.f, 0.f};
+              float acc[2][3][4];  // by K-step parity and 3xTF32 term: six independent chains
+#pragma unroll
+              for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int v = 0; v < 3; ++v)
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) acc[u][v][i] = 0.f;
               const float* la = Lf + (16 * a + g) * LDF + t4;
               const float* tb = Tf + t4 * LDT + 16 * b + n0 + g;
 #pragma unroll
@@ -671,11 +680,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int kk = 16 * b + 8 * ks;
                 const float af[4] = {la[kk], la[8 * LDF + kk], la[kk + 4], la[8 * LDF + kk + 4]};
                 const float bf[2] = {tb[kk * LDT], tb[(kk + 4) * LDT]};
-                mma_3xtf32(ym, yc, af, bf);
+                mma_3xtf32(acc[ks & 1], af, bf);
               }
               float y[4];
 #pragma unroll
-              for (int i = 0; i < 4; ++i) y[i] = ym[i] + yc[i];
+              for (int i = 0; i < 4; ++i)
+                y[i] = (acc[0][0][i] + acc[1][0][i]) + ((acc[0][1][i] + acc[1][1][i]) + (acc[0][2][i] + acc[1][2][i]));
               // Y[r][n] sits in lane 4 (r % 8) + n / 2, register 2 (r / 8) + n % 2; this lane needs
               // Y[t][g], Y[t+4][g] (first K step) and Y[8+t][g], Y[12+t][g] (second)
               const int s0 = 4 * t4 + (g >> 1), s1 = s0 + 16;
@@ -688,17 +698,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float u3 = __shfl_sync(0xffffffffu, y[2], s1), v3 = __shfl_sync(0xffffffffu, y[3], s1);
                 yb[0] = odd ? v0 : u0; yb[1] = odd ? v1 : u1; yb[2] = odd ? v2 : u2; yb[3] = odd ? v3 : u3;
               }
-              float om[4] = {0.f, 0.f, 0.f, 0.f}, oc[4] = {0.f, 0.f, 0.f, 0.f};
+              float oacc[2][3][4];
+#pragma unroll
+              for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int v = 0; v < 3; ++v)
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) oacc[u][v][i] = 0.f;
               const float* ta = Tf + (16 * a + g) * LDT + 16 * a + t4;
 #pragma unroll
               for (int ks = 0; ks < 2; ++ks) {
                 const float af[4] = {-ta[8 * ks], -ta[8 * LDT + 8 * ks], -ta[8 * ks + 4], -ta[8 * LDT + 8 * ks + 4]};
                 const float bf[2] = {yb[2 * ks], yb[2 * ks + 1]};
-                mma_3xtf32(om, oc, af, bf);
+                mma_3xtf32(oacc[ks], af, bf);
               }
+              float o4[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                o4[i] = (oacc[0][0][i] + oacc[1][0][i]) + ((oacc[0][1][i] + oacc[1][1][i]) + (oacc[0][2][i] + oacc[1][2][i]));
               float* to = Tf + (16 * a + g) * LDT + 16 * b + n0 + 2 * t4;
-              *reinterpret_cast<float2*>(to) = make_float2(om[0] + oc[0], om[1] + oc[1]);
-              *reinterpret_cast<float2*>(to + 8 * LDT) = make_float2(om[2] + oc[2], om[3] + oc[3]);
+              *reinterpret_cast<float2*>(to) = make_float2(o4[0], o4[1]);
+              *reinterpret_cast<float2*>(to + 8 * LDT) = make_float2(o4[2], o4[3]);
             }
             sync_wg();
           }
