@@ -413,84 +413,84 @@ __global__ void __launch_bounds__(kThreads, 1)
         op[oc] = pack8(f);
       }
     };
-    // bf16 copy of the state S for the UMMAs, then S <- Diag(e^{gamma_C}) S in TMEM, over the
-    // 32-column blocks [cb0, cb1) of this warp's 32 rows
-    auto state_copy = [&](int cb0, int cb1) {
-      const float ec = m->ec[row];
+    // bf16 copy of the state S for the UMMAs: 64-column halves [hb0, hb1) of this warp's 32 rows
+    auto state_copy = [&](int hb0, int hb1) {
 #pragma unroll 1
-      for (int cb = cb0; cb < cb1; ++cb) {
-        const int c0 = 32 * cb;
-        uint32_t v[32];
-        tmem_ld32(tl + TM_S + c0, v);
+      for (int hb = hb0; hb < hb1; ++hb) {
+        uint32_t v[64];
+        tmem_ld32(tl + TM_S + 64 * hb, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tl + TM_S + 64 * hb + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_wait_ld();
 #pragma unroll
-        for (int oc = 0; oc < 4; ++oc) {
+        for (int oc = 0; oc < 8; ++oc) {
           float f[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
-          at16(sm, OFF_S + sw128_oct(row, (c0 >> 3) + oc, 16384)) = pack8(f);
+          at16(sm, OFF_S + sw128_oct(row, 8 * hb + oc, 16384)) = pack8(f);
+        }
+      }
+    };
+
+    // thread of the decay scan and prep: channels 8o .. 8o+7, tokens t0 .. t0+3 of sub-tile b
+    const int qq = tid & 3, o = (tid >> 2) & 15, b = tid >> 6;
+    const int t0 = 16 * b + 4 * qq;
+    // Decay scan of one chunk (L tokens): gl = inclusive cumulative log2-decay from the start of
+    // the thread's sub-tile; se[m] = e^{decay over sub-tile m} per channel.
+    auto scan = [&](int L, float (&gl)[4][8]) {
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = t0 + i;
+        float g8[8];
+        if (t < L) {
+          unpack8(at16(sm, OFF_G + sw128_oct(t, o, 8192)), g8);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) g8[e] = 0.f;
         }
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) v[jj] = __float_as_uint(__uint_as_float(v[jj]) * ec);
-        tmem_st32(tl + TM_S + c0, v);
+        for (int e = 0; e < 8; ++e) {
+          if (checked && !(g8[e] >= KDA_G_MIN && g8[e] <= 0.f)) report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
+          acc[e] += g8[e] * kLog2e;
+          gl[i][e] = acc[e];
+        }
       }
-      tmem_wait_st();
+      // prefix over the four threads of the sub-tile (lanes differing in bits 0-1)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float x = acc[e];
+        float y = __shfl_up_sync(0xffffffffu, x, 1, 4);
+        if (qq >= 1) x += y;
+        y = __shfl_up_sync(0xffffffffu, x, 2, 4);
+        if (qq >= 2) x += y;
+        const float excl = x - acc[e];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) gl[i][e] += excl;
+        if (qq == 3) m->se[b][8 * o + e] = ex2(x);  // decay over the whole sub-tile
+      }
     };
 
     int L_prev = 0;
     int32_t tok_prev = 0;
+    float gl[4][8];  // the current chunk's decay scan
+    if (nchunks > 0) {  // the first chunk's scan; later ones run in the shadow of the previous chunk's UMMAs
+      ok = wg_wait(&m->full_g, 0);
+      if (ok) {
+        scan(min(C, seg.len), gl);
+        if (tid == 0) mbar_arrive(&m->empty_g);
+      }
+    }
     for (int j = 0; j < nchunks && ok; ++j) {
       const int L = min(C, seg.len - j * C);
       const int32_t tok = seg.tok0 + j * C;
       const uint32_t par = (uint32_t)(j & 1);
       const float* beta = m->beta[j & 1];
       if (write_out && j > 0) load_gate(L_prev, tok_prev);  // consumed by its epilogue below
-      if (!wg_wait(&m->full_g, par)) { ok = false; break; }
-
       // ---------------------------------------------------------------- decay prep: all bf16 operands
-      // thread: channels 8o .. 8o+7, tokens t0 .. t0+3 of sub-tile b
-      const int qq = tid & 3, o = (tid >> 2) & 15, b = tid >> 6;
-      const int t0 = 16 * b + 4 * qq;
-      float gl[4][8];     // inclusive cumulative log2-decay from the sub-tile start
-      {
-        float acc[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int t = t0 + i;
-          float g8[8];
-          if (t < L) {
-            unpack8(at16(sm, OFF_G + sw128_oct(t, o, 8192)), g8);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) g8[e] = 0.f;
-          }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            if (checked && !(g8[e] >= KDA_G_MIN && g8[e] <= 0.f)) report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
-            acc[e] += g8[e] * kLog2e;
-            gl[i][e] = acc[e];
-          }
-        }
-        // prefix over the four threads of the sub-tile (lanes differing in bits 0-1)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float x = acc[e];
-          float y = __shfl_up_sync(0xffffffffu, x, 1, 4);
-          if (qq >= 1) x += y;
-          y = __shfl_up_sync(0xffffffffu, x, 2, 4);
-          if (qq >= 2) x += y;
-          const float excl = x - acc[e];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) gl[i][e] += excl;
-          if (qq == 3) m->se[b][8 * o + e] = ex2(x);  // decay over the whole sub-tile
-        }
-      }
-      // g is consumed (its scan lives in registers): let the producer fetch the next chunk's g,
-      // then wait for this chunk's k and q
+
       if (!wg_wait(&m->full_kq, par)) { ok = false; break; }
-      if (tid == 0) mbar_arrive(&m->empty_g);
       // Per-channel factors, applied so that no O(1) value is multiplied by an underflowed
       // constant: with se_m = e^{decay over sub-tile m}, Eb = e^{r_b} = prod_{m<b} se_m, and per
       // token ix = e^{r_b - gamma_t} in [1, e^80]; the chain ix, ix se_b, ix se_b se_{b+1}, ...
@@ -649,10 +649,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int i = 0; i < 16; ++i) Tf[(o + i) * LDT + o + jc] = col[i];
         } else {
-          // meanwhile warps 2-7 copy and decay the state: warps 4 and 5 own TMEM lane quarters 0
-          // and 1 alone, warps 2|6 and 3|7 share quarters 2 and 3
-          if (q4 < 2) state_copy(0, 4);
-          else state_copy(warp < 4 ? 0 : 2, warp < 4 ? 2 : 4);
+          // meanwhile warps 2-7 make the bf16 copy of the state: warps 4 and 5 own TMEM lane
+          // quarters 0 and 1 alone, warps 2|6 and 3|7 share quarters 2 and 3
+          if (q4 < 2) state_copy(0, 2);
+          else state_copy(warp < 4 ? 0 : 1, warp < 4 ? 1 : 2);
         }
         sync_wg();
         // Off-diagonal blocks level by level (block distance d), one 16x8 strip per warp: warp
@@ -794,8 +794,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_k_loop(tmem + TM_WU, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S, 16384, false, 0, 8, id, false);
         umma_k_loop(tmem + TM_WU + hi, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S + 16384, 16384, false, 0, 8,
                     id, false);
+        umma_commit(&m->mma);
       }
-      if (!mma_commit_wait()) { ok = false; break; }
+      // in the shadow of these UMMAs (they read the bf16 copy of S, not TMEM columns [0,128)):
+      // S <- Diag(e^{gamma_C}) S in TMEM, then the next chunk's decay scan, whose g tile the
+      // producer fetched during this chunk; its release lets the producer fetch the one after
+      {
+        const float ec = m->ec[row];
+#pragma unroll
+        for (int hb = 0; hb < 2; ++hb) {
+          const int c0 = 64 * wg + 32 * hb;
+          uint32_t v[32];
+          tmem_ld32(tl + TM_S + c0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) v[jj] = __float_as_uint(__uint_as_float(v[jj]) * ec);
+          tmem_st32(tl + TM_S + c0, v);
+        }
+        tmem_wait_st();
+      }
+      bool next_ok = true;
+      if (j + 1 < nchunks) {
+        next_ok = wg_wait(&m->full_g, par ^ 1u);
+        if (next_ok) {
+          scan(min(C, seg.len - (j + 1) * C), gl);
+          if (tid == 0) mbar_arrive(&m->empty_g);
+        }
+      }
+      {
+        const bool r = wg_wait(&m->mma, mph & 1u);
+        ++mph;
+        tc_fence_after();
+        if (!r || !next_ok) { ok = false; break; }
+      }
       if (tid == 0) mbar_arrive(&m->empty_kq);  // k, q and their in-place products consumed
 
       // ---------------------------------------------------------------- U -> bf16 (same lane split as -W)
