@@ -26,12 +26,14 @@
 // handed back after the UMMAs that read their in-place products) and v (after W/U').  Warps 0-7
 // are two compute warpgroups; warp w owns TMEM lane quarter w % 4.  Decay prep, Gram read-out,
 // UT inverse and the -W / U conversions run on all 256 threads; in the shadow of the Gram UMMAs
-// both warpgroups run the previous chunk's epilogue, and while warps 0-1 invert the diagonal
-// blocks of the UT transform, warps 2-7 copy and decay the state.
-// Thread 0 issues the UMMAs.  The gate logits are staged from global memory with cp.async.
+// both warpgroups run the previous chunk's epilogue; while warps 0-1 invert the diagonal blocks
+// of the UT transform, warps 2-7 make the bf16 copy of the state; in the shadow of the U and O
+// UMMAs all warps decay the state and scan the next chunk's decay.  Off-diagonal blocks of the
+// inverse are warp-level tf32 MMAs.  Thread 0 issues the UMMAs.  The gate logits are staged
+// from global memory with cp.async.
 //
 // TMEM (512 columns allocated): [0,128) the fp32 state S (M=128; decayed in place while the
-// Gram UMMAs run, then K^T U accumulated onto it); [128,288) A|P (M=128, N = 16,32,48,64);
+// U and O UMMAs run, then K^T U accumulated onto it); [128,288) A|P (M=128, N=160);
 // [288,352) W -> O and [352,416) U' -> U: each M=64 product is issued as two N=64 halves, columns
 // 0-63 at lane offset 0 and columns 64-127 at lane offset 16 of the same TMEM columns, so a warp's
 // 32 lanes read 16 rows x 2 column halves and every lane takes part in the read-outs.
@@ -437,6 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Decay scan of one chunk (L tokens): gl = inclusive cumulative log2-decay from the start of
     // the thread's sub-tile; se[m] = e^{decay over sub-tile m} per channel.
     auto scan = [&](int L, float (&gl)[4][8]) {
+      bool bad = false;
       float acc[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -452,11 +455,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          if (checked && !(g8[e] >= KDA_G_MIN && g8[e] <= 0.f)) report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
+          bad |= !(g8[e] >= KDA_G_MIN && g8[e] <= 0.f);
           acc[e] += g8[e] * kLog2e;
           gl[i][e] = acc[e];
         }
       }
+      if (checked && bad) report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
       // prefix over the four threads of the sub-tile (lanes differing in bits 0-1)
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
