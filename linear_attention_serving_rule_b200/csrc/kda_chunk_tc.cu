@@ -89,7 +89,7 @@ struct Misc {
   uint32_t tmem_base;
   int32_t abort;
   float beta[2][C];  // double-buffered by chunk parity (written by the producer warp)
-  float se[4][DK];  // e^{decay over sub-tile m}, per channel
+  float se[4][DK];  // e^{decay over sub-tile m}; channel 8o + e at [m][16 e + o]
   float ec[DK];     // e^{gamma_C}
   float nw[DV];     // RMSNorm weight (1 without one)
   float ssq[2][C];  // epilogue: per-row sums of squares of the two column halves
@@ -433,8 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
 
-    // thread of the decay scan and prep: channels 8o .. 8o+7, tokens t0 .. t0+3 of sub-tile b
-    const int qq = tid & 3, o = (tid >> 2) & 15, b = tid >> 6;
+    // thread of the decay scan and prep: channels 8o .. 8o+7, tokens t0 .. t0+3 of sub-tile b.
+    // Eight consecutive lanes take eight channel octets of one token, so each quarter-warp's
+    // 16-byte accesses to a 128-byte swizzled tile hit eight distinct bank groups.
+    const int o = (lane & 7) + 8 * (warp & 1), qq = (lane >> 3) & 3, b = tid >> 6;
     const int t0 = 16 * b + 4 * qq;
     // Decay scan of one chunk (L tokens): gl = inclusive cumulative log2-decay from the start of
     // the thread's sub-tile; se[m] = e^{decay over sub-tile m} per channel.
@@ -461,18 +463,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (checked && bad) report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
-      // prefix over the four threads of the sub-tile (lanes differing in bits 0-1)
+      // prefix over the four threads of the sub-tile (lanes 8 apart)
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         float x = acc[e];
-        float y = __shfl_up_sync(0xffffffffu, x, 1, 4);
+        float y = __shfl_up_sync(0xffffffffu, x, 8);
         if (qq >= 1) x += y;
-        y = __shfl_up_sync(0xffffffffu, x, 2, 4);
+        y = __shfl_up_sync(0xffffffffu, x, 16);
         if (qq >= 2) x += y;
         const float excl = x - acc[e];
 #pragma unroll
         for (int i = 0; i < 4; ++i) gl[i][e] += excl;
-        if (qq == 3) m->se[b][8 * o + e] = ex2(x);  // decay over the whole sub-tile
+        if (qq == 3) m->se[b][16 * e + o] = ex2(x);  // decay over the whole sub-tile
       }
     };
 
@@ -506,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 8; ++e) {
           float se[4];
 #pragma unroll
-          for (int mm = 0; mm < 4; ++mm) se[mm] = m->se[mm][8 * o + e];
+          for (int mm = 0; mm < 4; ++mm) se[mm] = m->se[mm][16 * e + o];
           float eb = 1.f;
 #pragma unroll
           for (int mm = 0; mm < 4; ++mm)
@@ -568,7 +570,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           at16(sm, OFF_KH + sw128_oct(t, o, 8192)) = pack8(f);
         }
       }
-      if (tid < DK) m->ec[tid] = m->se[0][tid] * m->se[1][tid] * m->se[2][tid] * m->se[3][tid];
+      if (tid < DK) {
+        const int si = 16 * (tid & 7) + (tid >> 3);
+        m->ec[tid] = m->se[0][si] * m->se[1][si] * m->se[2][si] * m->se[3][si];
+      }
       sync_for_mma();
       // ---------------------------------------------------------------- UMMA: A | P
       if (tid == 0) {
