@@ -124,7 +124,27 @@ typedef struct kda_chunk_args {
   int32_t split_segments;
   void* workspace;
   size_t workspace_bytes;
+  float* snapshots;          /* [n_snap, H, dk, dv] float32 or NULL: chunk-boundary states */
+  int32_t snapshot_interval; /* tokens between snapshots: a positive multiple of 64 when
+                                snapshots != NULL (ignored otherwise) */
 } kda_chunk_args;
+
+/* Chunk-boundary state snapshots (prefix caching: a later call resumes a sequence from the state
+ * after any multiple of snapshot_interval tokens, passed as its initial_state).  The pages say that
+ * serving reuses earlier work because KDA carries a state instead of a token cache ("What's
+ * Actually Inside Kimi K3", section "Vision and Training") and that KDA makes prefix caching a new
+ * problem ("What's Kimi K3?", section "The Structure Beneath"); they give no interface.
+ *
+ * With I = snapshot_interval, sequence n (length len_n) gets snapshots after p = I, 2I, ...,
+ * floor(len_n / I) * I tokens: the state S_p of that sequence's recurrence, from its initial state,
+ * in the layout of final_state.  Snapshot p of sequence n is row base_n + p / I - 1 of `snapshots`,
+ * with base_n = sum over m < n of floor(len_m / I); n_snap = base_N.  A snapshot at p = len_n
+ * equals the final state.  The snapshot rows are written by kda_chunk_fwd; nothing else of the
+ * buffer is touched.  Errors: snapshots not 16-byte aligned, or I not a positive multiple of 64,
+ * -> KDA_ERR_INVALID_ARGUMENT.
+ * kda_chunk_fwd_snapshot_count stores n_snap (pure host computation; it reads num_seqs,
+ * total_tokens, cu_seqlens and snapshot_interval only, with the same checks as kda_chunk_fwd). */
+kda_status kda_chunk_fwd_snapshot_count(const kda_chunk_args* args, int64_t* n_snap);
 
 /* Bytes of workspace kda_chunk_fwd needs for these arguments (pure host computation). */
 kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args* args, size_t* bytes);

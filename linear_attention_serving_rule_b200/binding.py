@@ -36,7 +36,8 @@ KDA_FLAG_FORCE_SIMT = 0x2
 KDA_FLAG_TEST_FORCE_TIMEOUT = 0x4
 
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
-            "kda_read_device_error", "kda_status_string", "kda_chunk_fwd_noalloc")
+            "kda_read_device_error", "kda_status_string", "kda_chunk_fwd_noalloc",
+            "kda_chunk_fwd_snapshot_count")
 KDA_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 _P = ctypes.c_void_p
@@ -53,6 +54,7 @@ class KdaChunkArgs(ctypes.Structure):
         ("scale", ctypes.c_float), ("eps", ctypes.c_float), ("flags", ctypes.c_uint32),
         ("split_segments", ctypes.c_int32),
         ("workspace", _P), ("workspace_bytes", ctypes.c_size_t),
+        ("snapshots", _P), ("snapshot_interval", ctypes.c_int32),
     ]
 
 
@@ -90,6 +92,9 @@ def lib():
             L.kda_chunk_fwd_workspace_size.argtypes = [ctypes.POINTER(KdaChunkArgs),
                                                        ctypes.POINTER(ctypes.c_size_t)]
             L.kda_chunk_fwd_workspace_size.restype = ctypes.c_int
+            L.kda_chunk_fwd_snapshot_count.argtypes = [ctypes.POINTER(KdaChunkArgs),
+                                                       ctypes.POINTER(ctypes.c_int64)]
+            L.kda_chunk_fwd_snapshot_count.restype = ctypes.c_int
             L.kda_chunk_fwd.argtypes = [ctypes.POINTER(KdaChunkArgs), _P]
             L.kda_chunk_fwd.restype = ctypes.c_int
             L.kda_decode_step.argtypes = [ctypes.POINTER(KdaDecodeArgs), _P]
@@ -142,7 +147,7 @@ def _check_cuda(*ts):
 
 def make_chunk_args(q, k, v, g, beta, *, gate=None, cu_seqlens=None, initial_state=None,
                     norm_weight=None, out=None, final_state=None, scale=0.0, eps=1e-6,
-                    flags=0, split_segments=0, workspace=None):
+                    flags=0, split_segments=0, workspace=None, snapshots=None, snapshot_interval=0):
     """Fill a KdaChunkArgs.  Returns (args, keepalive) -- keep `keepalive` until the call."""
     keep = []
     if q.dim() == 4:
@@ -171,7 +176,27 @@ def make_chunk_args(q, k, v, g, beta, *, gate=None, cu_seqlens=None, initial_sta
     a.scale, a.eps, a.flags, a.split_segments = float(scale), float(eps), int(flags), int(split_segments)
     if workspace is not None:
         a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    a.snapshots, a.snapshot_interval = _ptr(snapshots), int(snapshot_interval)
     return a, keep
+
+
+def kda_chunk_fwd_snapshot_count(args: KdaChunkArgs) -> int:
+    n = ctypes.c_int64(0)
+    rc = lib().kda_chunk_fwd_snapshot_count(ctypes.byref(args), ctypes.byref(n))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd_snapshot_count")
+    return int(n.value)
+
+
+def snapshot_count(q, v, snapshot_interval, *, cu_seqlens=None) -> int:
+    """Rows of the snapshot buffer for these inputs (sum over sequences of len // interval)."""
+    if isinstance(cu_seqlens, torch.Tensor):
+        cu_seqlens = cu_seqlens.cpu().numpy()
+    a, keep = make_chunk_args(q, q, v, q, q, cu_seqlens=cu_seqlens, snapshot_interval=snapshot_interval)
+    # (the count reads the sequence layout and the interval only)
+    n = kda_chunk_fwd_snapshot_count(a)
+    del keep
+    return n
 
 
 def kda_chunk_fwd_workspace_size(args: KdaChunkArgs) -> int:
@@ -184,11 +209,14 @@ def kda_chunk_fwd_workspace_size(args: KdaChunkArgs) -> int:
 
 def kda_chunk_fwd(q, k, v, g, beta, *, gate=None, cu_seqlens=None, initial_state=None,
                   norm_weight=None, output_final_state=True, scale=0.0, eps=1e-6, flags=0,
-                  split_segments=0, out=None, final_state=None, workspace=None, stream=None):
+                  split_segments=0, out=None, final_state=None, workspace=None, stream=None,
+                  snapshots=None, snapshot_interval=0):
     """Chunkwise KDA prefill through the C ABI.
 
     q, k, g [T_tot, H, dk] (or [B, T, H, dk]); v, gate [.., H, dv]; beta [.., H];
     cu_seqlens: host sequence offsets (list / numpy / CPU tensor) for packed varlen input.
+    snapshots: optional fp32 [snapshot_count(...), H, dk, dv] buffer that receives the state after
+    every multiple of snapshot_interval tokens of every sequence (include/kda.h gives the rows).
     Returns (out, final_state, workspace).  Asynchronous on the current stream.
     """
     _check_cuda(q, k, v, g, beta, gate, initial_state, norm_weight)
@@ -203,7 +231,15 @@ def kda_chunk_fwd(q, k, v, g, beta, *, gate=None, cu_seqlens=None, initial_state
     a, keep = make_chunk_args(q, k, v, g, beta, gate=gate, cu_seqlens=cu_seqlens,
                               initial_state=initial_state, norm_weight=norm_weight, out=out,
                               final_state=final_state, scale=scale, eps=eps, flags=flags,
-                              split_segments=split_segments, workspace=workspace)
+                              split_segments=split_segments, workspace=workspace,
+                              snapshots=snapshots, snapshot_interval=snapshot_interval)
+    if snapshots is not None:
+        _check_cuda(snapshots)
+        need_rows = kda_chunk_fwd_snapshot_count(a)
+        if (snapshots.dtype != torch.float32 or not snapshots.is_contiguous()
+                or snapshots.numel() < need_rows * q.shape[-2] * q.shape[-1] * v.shape[-1]):
+            raise ValueError(f"snapshots must be a contiguous fp32 tensor of at least {need_rows} "
+                             f"x [H, dk, dv]")
     if workspace is None:
         need = kda_chunk_fwd_workspace_size(a)
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)

@@ -57,6 +57,10 @@ kda_status validate(const kda_chunk_args* a) {
   if (a->norm_weight && !aligned16(a->norm_weight)) return KDA_ERR_INVALID_ARGUMENT;
   if (a->initial_state && !aligned16(a->initial_state)) return KDA_ERR_INVALID_ARGUMENT;
   if (a->final_state && !aligned16(a->final_state)) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->snapshots) {
+    if (!aligned16(a->snapshots)) return KDA_ERR_INVALID_ARGUMENT;
+    if (a->snapshot_interval <= 0 || a->snapshot_interval % 64 != 0) return KDA_ERR_INVALID_ARGUMENT;
+  }
   if (a->cu_seqlens) {
     if (a->cu_seqlens[0] != 0) return KDA_ERR_INVALID_ARGUMENT;
     for (int32_t n = 0; n < a->num_seqs; ++n)
@@ -126,11 +130,38 @@ size_t workspace_bytes(const kda_chunk_args* a, const Layout& L) {
   return b;
 }
 
+Seg make_seg(int32_t t0, int32_t len, int32_t seq, int32_t role, int32_t slot, int32_t last) {
+  return Seg{t0, len, seq, role, slot, last, -1, 0};
+}
+
+// Snapshot rows: sequence n's snapshots start at row base[n] = sum_{m<n} floor(len_m / I).
+std::vector<int64_t> snapshot_bases(const Layout& L, int32_t I, int64_t* total) {
+  std::vector<int64_t> base(L.seqs.size());
+  int64_t acc = 0;
+  for (size_t n = 0; n < L.seqs.size(); ++n) {
+    base[n] = acc;
+    acc += L.seqs[n].len / I;
+  }
+  if (total) *total = acc;
+  return base;
+}
+
+// The first snapshot boundary inside a segment that starts q0 tokens into its sequence: the
+// smallest multiple of I above q0, if the segment reaches it.
+void assign_snapshot(Seg& s, int32_t q0, int32_t I, int64_t base) {
+  const int64_t p1 = ((int64_t)q0 / I + 1) * I;
+  const int64_t off = p1 - q0;
+  if (off <= s.len) {
+    s.snap = (int32_t)(base + p1 / I - 1);
+    s.snap_off = (int32_t)off;
+  }
+}
+
 // Launch `segs` (all of one role class) in batches of kPlanMax, longest first.
 cudaError_t run_segments(std::vector<Seg>& segs, const ChunkParams& p, kda_dtype dtype, bool use_tc,
                          cudaStream_t stream) {
   std::stable_sort(segs.begin(), segs.end(), [](const Seg& x, const Seg& y) { return x.len > y.len; });
-  static thread_local Plan plan;  // 24 KB: kept off the stack
+  static thread_local Plan plan;  // 30 KB: kept off the stack
   for (size_t b = 0; b < segs.size(); b += kPlanMax) {
     const size_t n = std::min<size_t>(kPlanMax, segs.size() - b);
     plan.n_seg = (int32_t)n;
@@ -146,6 +177,30 @@ cudaError_t run_segments(std::vector<Seg>& segs, const ChunkParams& p, kda_dtype
 }  // namespace kda
 
 using namespace kda;
+
+extern "C" kda_status kda_chunk_fwd_snapshot_count(const kda_chunk_args* a, int64_t* n_snap) {
+  // reads the sequence layout and the interval only
+  if (!a || !n_snap) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->num_seqs < 0 || a->total_tokens < 0) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->num_seqs == 0 && a->total_tokens != 0) return KDA_ERR_INVALID_ARGUMENT;
+  if (a->snapshot_interval <= 0 || a->snapshot_interval % 64 != 0) return KDA_ERR_INVALID_ARGUMENT;
+  int64_t n = 0;
+  for (int32_t i = 0; i < a->num_seqs; ++i) {
+    int64_t len;
+    if (a->cu_seqlens) {
+      if (a->cu_seqlens[i + 1] < a->cu_seqlens[i]) return KDA_ERR_INVALID_ARGUMENT;
+      len = a->cu_seqlens[i + 1] - a->cu_seqlens[i];
+    } else {
+      if (a->total_tokens % a->num_seqs != 0) return KDA_ERR_INVALID_ARGUMENT;
+      len = a->total_tokens / a->num_seqs;
+    }
+    n += len / a->snapshot_interval;
+  }
+  if (a->cu_seqlens && (a->cu_seqlens[0] != 0 || (int64_t)a->cu_seqlens[a->num_seqs] != a->total_tokens))
+    return KDA_ERR_INVALID_ARGUMENT;
+  *n_snap = n;
+  return KDA_OK;
+}
 
 extern "C" kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args* a, size_t* bytes) {
   if (!bytes) return KDA_ERR_INVALID_ARGUMENT;
@@ -170,6 +225,8 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
   p.out = a->out;
   p.final_state = a->final_state;
   p.error_word = (uint32_t*)a->workspace;
+  p.snapshots = a->snapshots;
+  p.snap_interval = a->snapshots ? a->snapshot_interval : 0;
   float* ws = (float*)((char*)a->workspace + kErrBytes);
   p.ws_state = L.slots ? ws : nullptr;
   p.ws_local = L.slots ? ws + (size_t)L.slots * a->H * a->dk * a->dv : nullptr;
@@ -189,11 +246,18 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
   // Pass 1 of split sequences: the head segment from the true initial state, and the
   // other non-final segments from [0 | I] (local state and transition matrix).
   std::vector<Seg> head, local, whole;
+  std::vector<int64_t> snap_base;
+  if (a->snapshots) snap_base = snapshot_bases(L, a->snapshot_interval, nullptr);
+  // segments that carry the true state write the snapshots inside them
+  auto with_snap = [&](Seg sg, int32_t n) {
+    if (a->snapshots) assign_snapshot(sg, sg.tok0 - L.seqs[n].tok0, a->snapshot_interval, snap_base[n]);
+    return sg;
+  };
   for (int32_t n = 0; n < a->num_seqs; ++n) {
     const SeqSpan& sp = L.seqs[n];
     const int32_t np = L.nseg[n];
     if (np == 1) {
-      whole.push_back({sp.tok0, sp.len, sp.seq, kRoleWhole, -1, 1});
+      whole.push_back(with_snap(make_seg(sp.tok0, sp.len, sp.seq, kRoleWhole, -1, 1), n));
       continue;
     }
     const int32_t sl = L.seglen[n], b = L.slot0[n];
@@ -201,17 +265,18 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
       const int32_t t0 = sp.tok0 + q * sl;
       const int32_t len = std::min(sl, sp.len - q * sl);
       if (q == 0) {
-        head.push_back({t0, len, sp.seq, kRoleHead, b, 0});
+        head.push_back(make_seg(t0, len, sp.seq, kRoleHead, b, 0));
       } else if (q < np - 1) {
         if (use_tc) {  // S_loc and M as two plain-state units of the tensor-core kernel
-          local.push_back({t0, len, sp.seq, kRoleLocalS, b + q, 0});
-          local.push_back({t0, len, sp.seq, kRoleLocalM, b + q, 0});
+          local.push_back(make_seg(t0, len, sp.seq, kRoleLocalS, b + q, 0));
+          local.push_back(make_seg(t0, len, sp.seq, kRoleLocalM, b + q, 0));
         } else {
-          local.push_back({t0, len, sp.seq, kRoleLocal, b + q, 0});
+          local.push_back(make_seg(t0, len, sp.seq, kRoleLocal, b + q, 0));
         }
       }
-      if (q == 0) whole.push_back({t0, len, sp.seq, kRoleWhole, b, 0});
-      else whole.push_back({t0, len, sp.seq, kRoleFromWs, b + q, q == np - 1 ? 1 : 0});
+      // the first segment's snapshots come from its pass-2 run (kRoleWhole from the initial state)
+      if (q == 0) whole.push_back(with_snap(make_seg(t0, len, sp.seq, kRoleWhole, b, 0), n));
+      else whole.push_back(with_snap(make_seg(t0, len, sp.seq, kRoleFromWs, b + q, q == np - 1 ? 1 : 0), n));
     }
   }
   cudaError_t e = cudaSuccess;
@@ -224,7 +289,7 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
     plan.n_seg = 0;
     for (int32_t n = 0; n < a->num_seqs && e == cudaSuccess; ++n) {
       if (L.nseg[n] <= 2) continue;
-      plan.seg[plan.n_seg++] = {L.seqs[n].tok0, L.nseg[n], L.seqs[n].seq, kRoleLocal, L.slot0[n], 0};
+      plan.seg[plan.n_seg++] = make_seg(L.seqs[n].tok0, L.nseg[n], L.seqs[n].seq, kRoleLocal, L.slot0[n], 0);
       if (plan.n_seg == kPlanMax) {
         e = launch_split_combine(plan, p, 0, stream);
         plan.n_seg = 0;

@@ -197,13 +197,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncthreads();
-    // ---- S = Diag(e^{gamma_C}) S0 + (k e^{gamma_C - gamma})^T U
+    // ---- S = Diag(e^{gamma_C}) S0 + (k e^{gamma_C - gamma})^T U; a chunk that ends on a snapshot
+    // boundary also writes S to its snapshot row
+    float* snap = nullptr;
+    {
+      const int e = c0 + L;
+      if (seg.snap >= 0 && e >= seg.snap_off && (e - seg.snap_off) % p.snap_interval == 0)
+        snap = p.snapshots + ((size_t)(seg.snap + (e - seg.snap_off) / p.snap_interval) * H + h) * (size_t)(DK * DV);
+    }
     for (int idx = tid; idx < DK * NS; idx += kThreads) {
       const int i = idx / NS, j = idx - i * NS;
       float acc = sm.eC[i] * sm.S[idx];
 #pragma unroll
       for (int t = 0; t < kC; ++t) acc += sm.Kh[t * DK + i] * sm.U[t * NS + j];
       sm.S[idx] = acc;
+      if (snap && j < DV) snap[i * DV + j] = acc;
     }
     // ---- epilogue: head-wise RMSNorm * sigmoid(gate), one warp per token
     if (write_out) {

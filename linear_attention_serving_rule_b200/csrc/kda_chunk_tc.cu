@@ -99,6 +99,8 @@ static_assert(sizeof(Misc) <= 8192, "misc block too large");
 struct TcMaps {
   CUtensorMap q, k, g, v;
 };
+static_assert(sizeof(Plan) + sizeof(TcMaps) + sizeof(ChunkParams) + 128 <= 32764,
+              "kernel parameters exceed the 32,764-byte limit");
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
@@ -295,6 +297,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
     const size_t unit_state = (size_t)DK * DV;
     const bool write_out = (seg.role == kRoleWhole || seg.role == kRoleFromWs);
+    // chunk-boundary snapshot of the state after segment-local token e, or null
+    auto snap_dst = [&](int e) -> float* {
+      if (seg.snap < 0 || e < seg.snap_off || (e - seg.snap_off) % p.snap_interval != 0) return nullptr;
+      const int row_s = seg.snap + (e - seg.snap_off) / p.snap_interval;
+      return p.snapshots + ((size_t)row_s * H + h) * unit_state;
+    };
     uint32_t mph = 0;
     bool ok = true;
 
@@ -415,14 +423,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         op[oc] = pack8(f);
       }
     };
-    // bf16 copy of the state S for the UMMAs: 64-column halves [hb0, hb1) of this warp's 32 rows
-    auto state_copy = [&](int hb0, int hb1) {
+    // bf16 copy of the state S for the UMMAs: 64-column halves [hb0, hb1) of this warp's 32 rows;
+    // with snap != null also the fp32 snapshot of S
+    auto state_copy = [&](int hb0, int hb1, float* snap) {
 #pragma unroll 1
       for (int hb = hb0; hb < hb1; ++hb) {
         uint32_t v[64];
         tmem_ld32(tl + TM_S + 64 * hb, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
         tmem_ld32(tl + TM_S + 64 * hb + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
         tmem_wait_ld();
+        if (snap) {
+          float4* d4 = reinterpret_cast<float4*>(snap + (size_t)row * DV + 64 * hb);
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj)
+            d4[jj] = make_float4(__uint_as_float(v[4 * jj]), __uint_as_float(v[4 * jj + 1]),
+                                 __uint_as_float(v[4 * jj + 2]), __uint_as_float(v[4 * jj + 3]));
+        }
 #pragma unroll
         for (int oc = 0; oc < 8; ++oc) {
           float f[8];
@@ -660,8 +676,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           // meanwhile warps 2-7 make the bf16 copy of the state: warps 4 and 5 own TMEM lane
           // quarters 0 and 1 alone, warps 2|6 and 3|7 share quarters 2 and 3
-          if (q4 < 2) state_copy(0, 2);
-          else state_copy(warp < 4 ? 0 : 1, warp < 4 ? 1 : 2);
+          // (the state here is the one after the previous chunk: a snapshot if that chunk ended
+          // on a snapshot boundary)
+          float* snap = j > 0 ? snap_dst(j * C) : nullptr;
+          if (q4 < 2) state_copy(0, 2, snap);
+          else state_copy(warp < 4 ? 0 : 1, warp < 4 ? 1 : 2, snap);
         }
         sync_wg();
         // Off-diagonal blocks level by level (block distance d), one 16x8 strip per warp: warp
@@ -889,7 +908,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         ld = DV + DK;
         dst = p.ws_local + ((size_t)seg.slot * H + h) * (size_t)DK * ld + (seg.role == kRoleLocalM ? DV : 0);
       }
-      if (dst) {
+      float* sdst = nchunks > 0 ? snap_dst(seg.len) : nullptr;  // a snapshot boundary at the segment end
+      if (dst || sdst) {
 #pragma unroll
         for (int hb = 0; hb < 2; ++hb) {
           const int c0 = wg * 64 + hb * 32;
@@ -897,10 +917,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld32(tl + TM_S + c0, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int jj = 0; jj < 32; jj += 4)
-            *reinterpret_cast<float4*>(dst + (size_t)row * ld + c0 + jj) =
-                make_float4(__uint_as_float(v[jj]), __uint_as_float(v[jj + 1]), __uint_as_float(v[jj + 2]),
-                            __uint_as_float(v[jj + 3]));
+          for (int jj = 0; jj < 32; jj += 4) {
+            const float4 x = make_float4(__uint_as_float(v[jj]), __uint_as_float(v[jj + 1]),
+                                         __uint_as_float(v[jj + 2]), __uint_as_float(v[jj + 3]));
+            if (dst) *reinterpret_cast<float4*>(dst + (size_t)row * ld + c0 + jj) = x;
+            if (sdst) *reinterpret_cast<float4*>(sdst + (size_t)row * DV + c0 + jj) = x;
+          }
         }
       }
     } else if (tid == 0 && mph > 0) {

@@ -14,7 +14,8 @@
 
 namespace kda {
 
-constexpr int kPlanMax = 1024;  // segments per launch (the plan travels in the kernel parameters)
+constexpr int kPlanMax = 960;  // segments per launch (the plan travels in the kernel parameters,
+                               // which hold at most 32,764 bytes)
 
 // Where a unit's start state comes from and where its end state goes.
 enum SegRole : int32_t {
@@ -38,6 +39,8 @@ struct Seg {
   int32_t role;   // SegRole
   int32_t slot;   // workspace slot (split passes), -1 if unused
   int32_t last;   // 1 if this segment ends its sequence (writes final_state)
+  int32_t snap;      // snapshot row of the first snapshot boundary inside the segment, -1 if none
+  int32_t snap_off;  // that boundary's offset from the segment start, in tokens (1 .. len)
 };
 
 struct Plan {
@@ -61,6 +64,8 @@ struct ChunkParams {
   float* ws_state;     // split: per-slot [dk, dv] start states (pass 2 reads), or null
   float* ws_local;     // split: per-slot [dk, dv + dk] (S_loc | M) from pass 1, or null
   uint32_t* error_word;
+  float* snapshots;      // [n_snap, H, dk, dv] chunk-boundary states, or null
+  int32_t snap_interval; // tokens between snapshot boundaries (a multiple of 64)
   int64_t total_tokens;  // rows of the packed tensors (tensor-map extent)
   int32_t H, dk, dv;
   float scale, eps;

@@ -48,6 +48,8 @@ def _bind(path):
         P, P, P, P, P, P, P, P, ctypes.c_double, ctypes.c_double,
         ctypes.c_uint32, ctypes.c_int32, P, P]
     lib.kda_ref_forward.restype = ctypes.c_int
+    lib.kda_ref_forward_snapshots.argtypes = lib.kda_ref_forward.argtypes + [ctypes.c_int64, P]
+    lib.kda_ref_forward_snapshots.restype = ctypes.c_int
     lib.kda_ref_decode_step.argtypes = [
         ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
         P, P, P, P, P, P, P, P, P, ctypes.c_double, ctypes.c_double,
@@ -79,6 +81,9 @@ class Oracle:
 
     def forward(self, *a, **kw):
         return forward(*a, _lib=self._l(), **kw)
+
+    def forward_snapshots(self, *a, **kw):
+        return forward_snapshots(*a, _lib=self._l(), **kw)
 
     def decode_step(self, *a, **kw):
         return decode_step(*a, _lib=self._l(), **kw)
@@ -117,7 +122,7 @@ def max_threads() -> int:
 
 def forward(q, k, v, g, beta, *, cu_seqlens=None, gate=None, norm_weight=None,
             initial_state=None, scale=None, eps=1e-6, mode=0, num_threads=0,
-            return_final_state=True, _lib=None):
+            return_final_state=True, _lib=None, _snapshot_interval=None):
     """Run the oracle over a packed batch.
 
     q, k, g: [T_tot, H, dk]; v, gate: [T_tot, H, dv]; beta: [T_tot, H] (any
@@ -150,15 +155,32 @@ def forward(q, k, v, g, beta, *, cu_seqlens=None, gate=None, norm_weight=None,
     fin = np.zeros((N, H, dk, dv), dtype=np.float64) if return_final_state else None
     if scale is None:
         scale = 1.0 / np.sqrt(dk)
-    rc = (_lib or _load()).kda_ref_forward(N, _ptr(cu), H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(g),
-                                 _ptr(beta), _ptr(gate), _ptr(norm_weight), _ptr(S0),
-                                 float(scale), float(eps), int(mode), int(num_threads),
-                                 _ptr(out), _ptr(fin))
+    args = (N, _ptr(cu), H, dk, dv, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(gate),
+            _ptr(norm_weight), _ptr(S0), float(scale), float(eps), int(mode), int(num_threads),
+            _ptr(out), _ptr(fin))
+    snaps = None
+    if _snapshot_interval is None:
+        rc = (_lib or _load()).kda_ref_forward(*args)
+    else:
+        I = int(_snapshot_interval)
+        if I <= 0:
+            raise ValueError("snapshot_interval must be positive")
+        rows = int(sum((int(cu[n + 1]) - int(cu[n])) // I for n in range(N)))
+        snaps = np.zeros((max(rows, 1), H, dk, dv), dtype=np.float64)
+        rc = (_lib or _load()).kda_ref_forward_snapshots(*args, I, _ptr(snaps))
+        snaps = snaps[:rows]
     if rc != 0:
         raise ValueError(f"kda_ref_forward rejected its arguments (rc={rc})")
     if dense:
         out = out.reshape(B, T, H, dv)
-    return out, fin
+    return (out, fin) if snaps is None else (out, fin, snaps)
+
+
+def forward_snapshots(q, k, v, g, beta, snapshot_interval, **kw):
+    """forward() that also returns the state after every multiple of snapshot_interval tokens of
+    each sequence: (out, final_state, snapshots [rows, H, dk, dv] float64), rows ordered by
+    sequence, then by position (the layout kda_ref.h gives)."""
+    return forward(q, k, v, g, beta, _snapshot_interval=snapshot_interval, **kw)
 
 
 def decode_step(q, k, v, g, beta, state, *, gate=None, norm_weight=None,

@@ -82,14 +82,19 @@ static int check_common(int32_t H, int32_t dk, int32_t dv, const float* q,
   return KDA_REF_OK;
 }
 
-int kda_ref_forward(int64_t num_seqs, const int64_t* cu_seqlens, int32_t H,
-                    int32_t dk, int32_t dv, const float* q, const float* k,
-                    const float* v, const float* g, const float* beta,
-                    const float* gate, const float* norm_weight,
-                    const double* initial_state, double scale, double eps,
-                    uint32_t mode, int32_t num_threads, double* out,
-                    double* final_state) {
+/* The sequential recurrence over every (sequence, head) unit; with snapshots != NULL the state
+ * after each multiple of snapshot_interval tokens of a sequence is also copied out (the state
+ * S_p of the definition, nothing else). */
+static int forward_impl(int64_t num_seqs, const int64_t* cu_seqlens, int32_t H,
+                        int32_t dk, int32_t dv, const float* q, const float* k,
+                        const float* v, const float* g, const float* beta,
+                        const float* gate, const float* norm_weight,
+                        const double* initial_state, double scale, double eps,
+                        uint32_t mode, int32_t num_threads, double* out,
+                        double* final_state, int64_t snapshot_interval,
+                        double* snapshots) {
   if (num_seqs < 0 || !cu_seqlens || !out) return KDA_REF_BAD_ARG;
+  if (snapshots && snapshot_interval <= 0) return KDA_REF_BAD_ARG;
   if (check_common(H, dk, dv, q, k, v, g, beta)) return KDA_REF_BAD_ARG;
   if (cu_seqlens[0] != 0) return KDA_REF_BAD_ARG;
   for (int64_t n = 0; n < num_seqs; ++n)
@@ -98,6 +103,15 @@ int kda_ref_forward(int64_t num_seqs, const int64_t* cu_seqlens, int32_t H,
   const int64_t units = num_seqs * (int64_t)H;
   const size_t state_elems = (size_t)dk * (size_t)dv;
   int bad = 0;
+  /* snapshot row of sequence n's first snapshot: sum over m < n of floor(len_m / interval) */
+  int64_t* snap_base = NULL;
+  if (snapshots) {
+    snap_base = (int64_t*)malloc(sizeof(int64_t) * (size_t)(num_seqs + 1));
+    if (!snap_base) return KDA_REF_BAD_ARG;
+    snap_base[0] = 0;
+    for (int64_t n = 0; n < num_seqs; ++n)
+      snap_base[n + 1] = snap_base[n] + (cu_seqlens[n + 1] - cu_seqlens[n]) / snapshot_interval;
+  }
 #ifdef _OPENMP
   if (num_threads > 0) omp_set_num_threads(num_threads);
 #else
@@ -128,6 +142,12 @@ int kda_ref_forward(int64_t num_seqs, const int64_t* cu_seqlens, int32_t H,
         token_step(dk, dv, S, q + row * dk, k + row * dk, v + row * dv,
                    g + row * dk, (double)beta[row], scale, mode, u, o);
         if (gate) rmsnorm_gate(dv, o, gate + row * dv, norm_weight, eps);
+        const int64_t done = t - cu_seqlens[n] + 1; /* tokens of the sequence consumed */
+        if (snapshots && done % snapshot_interval == 0) {
+          const int64_t srow = snap_base[n] + done / snapshot_interval - 1;
+          memcpy(snapshots + ((size_t)srow * H + h) * state_elems, S,
+                 sizeof(double) * state_elems);
+        }
       }
       if (final_state)
         memcpy(final_state + (size_t)unit * state_elems, S,
@@ -136,7 +156,34 @@ int kda_ref_forward(int64_t num_seqs, const int64_t* cu_seqlens, int32_t H,
     free(S);
     free(u);
   }
+  free(snap_base);
   return bad ? KDA_REF_BAD_ARG : KDA_REF_OK;
+}
+
+int kda_ref_forward(int64_t num_seqs, const int64_t* cu_seqlens, int32_t H,
+                    int32_t dk, int32_t dv, const float* q, const float* k,
+                    const float* v, const float* g, const float* beta,
+                    const float* gate, const float* norm_weight,
+                    const double* initial_state, double scale, double eps,
+                    uint32_t mode, int32_t num_threads, double* out,
+                    double* final_state) {
+  return forward_impl(num_seqs, cu_seqlens, H, dk, dv, q, k, v, g, beta, gate,
+                      norm_weight, initial_state, scale, eps, mode, num_threads,
+                      out, final_state, 0, NULL);
+}
+
+int kda_ref_forward_snapshots(int64_t num_seqs, const int64_t* cu_seqlens, int32_t H,
+                              int32_t dk, int32_t dv, const float* q, const float* k,
+                              const float* v, const float* g, const float* beta,
+                              const float* gate, const float* norm_weight,
+                              const double* initial_state, double scale, double eps,
+                              uint32_t mode, int32_t num_threads, double* out,
+                              double* final_state, int64_t snapshot_interval,
+                              double* snapshots) {
+  if (!snapshots) return KDA_REF_BAD_ARG;
+  return forward_impl(num_seqs, cu_seqlens, H, dk, dv, q, k, v, g, beta, gate,
+                      norm_weight, initial_state, scale, eps, mode, num_threads,
+                      out, final_state, snapshot_interval, snapshots);
 }
 
 int kda_ref_decode_step(int64_t N, int32_t H, int32_t dk, int32_t dv,

@@ -64,6 +64,19 @@ int kda_ref_forward(int64_t num_seqs, const int64_t* cu_seqlens, int32_t H,
                     uint32_t mode, int32_t num_threads, double* out,
                     double* final_state);
 
+/* kda_ref_forward, and also the state after every multiple of snapshot_interval
+ * tokens of each sequence: snapshot p of sequence n (p = I, 2I, .., floor(len_n/I) I)
+ * is row base_n + p/I - 1 of snapshots [rows, H, dk, dv], base_n = sum_{m<n}
+ * floor(len_m / I).  The state S_p is the recurrence's own state after token p. */
+int kda_ref_forward_snapshots(int64_t num_seqs, const int64_t* cu_seqlens, int32_t H,
+                              int32_t dk, int32_t dv, const float* q, const float* k,
+                              const float* v, const float* g, const float* beta,
+                              const float* gate, const float* norm_weight,
+                              const double* initial_state, double scale, double eps,
+                              uint32_t mode, int32_t num_threads, double* out,
+                              double* final_state, int64_t snapshot_interval,
+                              double* snapshots);
+
 /* One decode step: one new token per sequence.  Inputs are [N, H, d];
  * state is [num_slots, H, dk, dv] updated in place; sequence n uses slot
  * state_indices[n] (or n when state_indices is NULL). */

@@ -168,3 +168,38 @@ def test_decode_validation(L):
     assert f(N=-1) == B.KDA_ERR_INVALID_ARGUMENT
     assert f(N=0) == B.KDA_OK                                  # nothing to do, nothing launched
     assert L.kda_read_device_error(None, None) == B.KDA_ERR_INVALID_ARGUMENT
+
+
+def _count(L, a):
+    n = ctypes.c_int64(-1)
+    rc = L.kda_chunk_fwd_snapshot_count(ctypes.byref(a), ctypes.byref(n))
+    return rc, n.value
+
+
+def test_snapshot_arguments(L):
+    # a snapshot buffer needs 16-byte alignment and an interval that is a positive multiple of 64
+    assert _fwd(L, _args(snapshots=FAKE + 8, snapshot_interval=64)) == B.KDA_ERR_INVALID_ARGUMENT
+    for bad in (0, -64, 32, 96):
+        assert _fwd(L, _args(snapshots=FAKE, snapshot_interval=bad)) == B.KDA_ERR_INVALID_ARGUMENT
+        assert _count(L, _args(snapshot_interval=bad))[0] == B.KDA_ERR_INVALID_ARGUMENT
+    # without a buffer the interval is ignored
+    assert _ws(L, _args(snapshots=None, snapshot_interval=32))[0] == B.KDA_OK
+
+
+def test_snapshot_count(L):
+    # sum over sequences of floor(len / interval); zero-length and short sequences contribute 0
+    cu = np.array([0, 100, 300, 300, 1000], dtype=np.int32)
+    a = _args(num_seqs=4, total_tokens=1000, cu_seqlens=cu.ctypes.data)
+    for I, want in ((64, 1 + 3 + 0 + 10), (128, 0 + 1 + 0 + 5), (1024, 0)):
+        a.snapshot_interval = I
+        assert _count(L, a) == (B.KDA_OK, want)
+    # dense batch: 2 sequences of 128 tokens
+    assert _count(L, _args(snapshot_interval=64)) == (B.KDA_OK, 4)
+    assert _count(L, _args(snapshot_interval=128)) == (B.KDA_OK, 2)
+    # only the layout and the interval are read: no tensor pointers needed
+    bare = B.KdaChunkArgs()
+    bare.num_seqs, bare.total_tokens, bare.cu_seqlens, bare.snapshot_interval = 4, 1000, cu.ctypes.data, 64
+    assert _count(L, bare) == (B.KDA_OK, 14)
+    bad = np.array([0, 100, 90, 1000], dtype=np.int32)
+    assert _count(L, _args(num_seqs=3, total_tokens=1000, cu_seqlens=bad.ctypes.data,
+                           snapshot_interval=64))[0] == B.KDA_ERR_INVALID_ARGUMENT

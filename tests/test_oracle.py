@@ -145,6 +145,37 @@ def pin_unrolled_transition_product(ref, seed=4):
     np.testing.assert_allclose(fin[0, 0], St, rtol=1e-11, atol=1e-12)
 
 
+# --- I3b: chunk-boundary snapshots are the unrolled prefix states -------------------------------
+def pin_snapshots_are_unrolled_prefix_states(ref, seed=7):
+    """Snapshot p of a sequence is S_p = (prod_{r<p} M_r) S0 + sum_{t<p} (prod_{t<r<p} M_r)
+    beta_t k_t v_t^T, computed here from the dense transition matrices for every boundary of two
+    ragged sequences (lengths 130 and 70, interval 64), each head with its own initial state."""
+    rng = _rng(seed)
+    lens, H, dk, dv, I = (130, 70), 2, 3, 2, 64
+    Tt = sum(lens)
+    cu = np.array([0, lens[0], Tt], dtype=np.int64)
+    q = rng.standard_normal((Tt, H, dk)).astype(np.float32)
+    k = rng.standard_normal((Tt, H, dk)).astype(np.float32)
+    v = rng.standard_normal((Tt, H, dv)).astype(np.float32)
+    g = (-0.05 * rng.random((Tt, H, dk))).astype(np.float32)  # slow decay: early tokens still count
+    beta = rng.random((Tt, H)).astype(np.float32)
+    s0 = rng.standard_normal((2, H, dk, dv))
+    out, fin, snaps = ref.forward_snapshots(q, k, v, g, beta, I, cu_seqlens=cu, initial_state=s0)
+    assert snaps.shape == (lens[0] // I + lens[1] // I, H, dk, dv)
+    row = 0
+    for n in range(2):
+        for p_ in range(I, lens[n] + 1, I):
+            for h in range(H):
+                S = s0[n, h].copy()
+                for t in range(cu[n], cu[n] + p_):
+                    kk = k[t, h].astype(np.float64)
+                    M = (np.eye(dk) - float(beta[t, h]) * np.outer(kk, kk)) @ np.diag(np.exp(g[t, h].astype(np.float64)))
+                    S = M @ S + float(beta[t, h]) * np.outer(kk, v[t, h].astype(np.float64))
+                np.testing.assert_allclose(snaps[row, h], S, rtol=1e-10, atol=1e-12)
+            row += 1
+    assert row == snaps.shape[0]
+
+
 # --- I4: orthonormal keys form an exact associative memory ----------------------------------
 def pin_orthonormal_keys_are_recalled_exactly(ref):
     """g = 0, beta = 1, keys = distinct rows of a normalised 16x16 Hadamard matrix (exactly
@@ -287,7 +318,8 @@ PINS = [pin_delta_write_is_exact_for_unit_keys, pin_beta_zero_is_pure_decay,
         pin_erase_off_equals_gated_linear_attention, pin_unrolled_transition_product,
         pin_orthonormal_keys_are_recalled_exactly, pin_linear_in_values_and_initial_state,
         pin_split_invariance_and_varlen_packing, pin_epilogue_matches_library_rmsnorm,
-        pin_decode_step_matches_one_token_forward, pin_scalar_worked_example]
+        pin_decode_step_matches_one_token_forward, pin_scalar_worked_example,
+        pin_snapshots_are_unrolled_prefix_states]
 
 
 @pytest.fixture(scope="module")

@@ -29,6 +29,9 @@ MUTANTS = [
     ("readout_before_write", None, None),   # built below: the read-out moved before the write
     ("decode_ignores_slot_map", "const int64_t slot = state_indices ? state_indices[n] : n;",
      "const int64_t slot = n;"),
+    ("snapshot_wrong_head", "memcpy(snapshots + ((size_t)srow * H + h) * state_elems, S,",
+     "memcpy(snapshots + ((size_t)srow * H + 0) * state_elems, S,"),
+    ("snapshot_one_token_early", None, None),  # built below: the copy moved before the token's update
 ]
 
 
@@ -54,6 +57,13 @@ def _mutant_source(name, old, new):
         src = src[:i] + src[j:]
         k = src.index("  for (int32_t i = 0; i < dk; ++i) {\n    const double ki = (double)k[i];\n    double* row")
         return src[:k] + readout + src[k:]
+    if name == "snapshot_one_token_early":
+        i, j = _block(src, "        const int64_t done = t - cu_seqlens[n] + 1;",
+                      "sizeof(double) * state_elems);\n        }\n")
+        snap = src[i:j]
+        src = src[:i] + src[j:]
+        k = src.index("        token_step(dk, dv, S, q + row * dk, k + row * dk, v + row * dv,")
+        return src[:k] + snap + src[k:]
     assert old in src, f"mutation anchor for {name} not found"
     return src.replace(old, new, 1)
 
