@@ -26,6 +26,9 @@ _lock = threading.Lock()
 _lib = None
 
 ERASE_OFF = 1
+G_LOGITS = 2       # g holds decay logits a: g = -5 sigmoid(a)
+BETA_LOGITS = 4    # beta holds logits: beta = sigmoid(b)
+QK_L2NORM = 8      # q, k L2-normalised per (token, head): x / sqrt(sum x^2 + 1e-6)
 
 
 def build(force: bool = False) -> str:
@@ -72,6 +75,7 @@ class Oracle:
     """The oracle bound to one compiled library (the default one, or a test's variant)."""
 
     ERASE_OFF = ERASE_OFF
+    G_LOGITS, BETA_LOGITS, QK_L2NORM = G_LOGITS, BETA_LOGITS, QK_L2NORM
 
     def __init__(self, lib_path=None):
         self._lib = _bind(lib_path) if lib_path else None

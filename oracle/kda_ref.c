@@ -42,8 +42,8 @@ static void rmsnorm_gate(int32_t dv, double* o, const float* gate,
  *   3. write:   S += k u^T
  *   4. read:    o = scale * S^T q             (after the write)
  * Steps 1-3 equal S_t = (I - beta k k^T) Diag(e^g) S_{t-1} + beta k v^T. */
-static void token_step(int32_t dk, int32_t dv, double* S, const float* q,
-                       const float* k, const float* v, const float* g,
+static void token_step(int32_t dk, int32_t dv, double* S, const double* q,
+                       const double* k, const float* v, const double* g,
                        double beta, double scale, uint32_t mode, double* u,
                        double* o) {
   for (int32_t i = 0; i < dk; ++i) {
@@ -72,6 +72,39 @@ static void token_step(int32_t dk, int32_t dv, double* S, const float* q,
     for (int32_t j = 0; j < dv; ++j) o[j] += row[j] * qi;
   }
   for (int32_t j = 0; j < dv; ++j) o[j] *= scale;
+}
+
+/* The token's q, k, g and beta as the recurrence uses them, in double.  With the
+ * pre-processing mode bits the inputs are the raw projections instead:
+ *   KDA_REF_G_LOGITS:    g = g_min * sigmoid(a), g_min = -5 (the scaled-sigmoid
+ *                        decay: "Kimi K3: Engineering a 2.8 Trillion Parameter
+ *                        Frontier", section "Dimension 1"; "Kimi K3 Architecture
+ *                        Explained", section "Token mixing")
+ *   KDA_REF_BETA_LOGITS: beta = sigmoid(b)
+ *   KDA_REF_QK_L2NORM:   q <- q / sqrt(sum_i q_i^2 + 1e-6), the same for k
+ *                        (unit-norm keys are what makes the delta write a
+ *                        Householder projection: "Kimi K3 de Moonshot AI",
+ *                        section "Kimi Delta Attention (KDA)") */
+static double prep_token(int32_t dk, const float* q, const float* k, const float* g,
+                         float beta, uint32_t mode, double* qd, double* kd, double* gd) {
+  for (int32_t i = 0; i < dk; ++i) {
+    qd[i] = (double)q[i];
+    kd[i] = (double)k[i];
+    gd[i] = (mode & KDA_REF_G_LOGITS) ? KDA_REF_G_MIN * sigmoid((double)g[i]) : (double)g[i];
+  }
+  if (mode & KDA_REF_QK_L2NORM) {
+    double sq = 0.0, sk = 0.0;
+    for (int32_t i = 0; i < dk; ++i) {
+      sq += qd[i] * qd[i];
+      sk += kd[i] * kd[i];
+    }
+    const double rq = 1.0 / sqrt(sq + KDA_REF_L2NORM_EPS), rk = 1.0 / sqrt(sk + KDA_REF_L2NORM_EPS);
+    for (int32_t i = 0; i < dk; ++i) {
+      qd[i] *= rq;
+      kd[i] *= rk;
+    }
+  }
+  return (mode & KDA_REF_BETA_LOGITS) ? sigmoid((double)beta) : (double)beta;
 }
 
 static int check_common(int32_t H, int32_t dk, int32_t dv, const float* q,
@@ -122,13 +155,14 @@ static int forward_impl(int64_t num_seqs, const int64_t* cu_seqlens, int32_t H,
   {
     double* S = (double*)malloc(sizeof(double) * state_elems);
     double* u = (double*)malloc(sizeof(double) * (size_t)dv);
-    if (!S || !u) {
+    double* qkg = (double*)malloc(sizeof(double) * 3 * (size_t)dk);
+    if (!S || !u || !qkg) {
 #pragma omp atomic write
       bad = 1;
     }
 #pragma omp for schedule(dynamic, 1)
     for (int64_t unit = 0; unit < units; ++unit) {
-      if (!S || !u) continue;
+      if (!S || !u || !qkg) continue;
       const int64_t n = unit / H;
       const int32_t h = (int32_t)(unit % H);
       if (initial_state)
@@ -139,8 +173,9 @@ static int forward_impl(int64_t num_seqs, const int64_t* cu_seqlens, int32_t H,
       for (int64_t t = cu_seqlens[n]; t < cu_seqlens[n + 1]; ++t) {
         const size_t row = (size_t)t * H + h;
         double* o = out + row * dv;
-        token_step(dk, dv, S, q + row * dk, k + row * dk, v + row * dv,
-                   g + row * dk, (double)beta[row], scale, mode, u, o);
+        const double b = prep_token(dk, q + row * dk, k + row * dk, g + row * dk, beta[row],
+                                    mode, qkg, qkg + dk, qkg + 2 * dk);
+        token_step(dk, dv, S, qkg, qkg + dk, v + row * dv, qkg + 2 * dk, b, scale, mode, u, o);
         if (gate) rmsnorm_gate(dv, o, gate + row * dv, norm_weight, eps);
         const int64_t done = t - cu_seqlens[n] + 1; /* tokens of the sequence consumed */
         if (snapshots && done % snapshot_interval == 0) {
@@ -155,6 +190,7 @@ static int forward_impl(int64_t num_seqs, const int64_t* cu_seqlens, int32_t H,
     }
     free(S);
     free(u);
+    free(qkg);
   }
   free(snap_base);
   return bad ? KDA_REF_BAD_ARG : KDA_REF_OK;
@@ -204,24 +240,27 @@ int kda_ref_decode_step(int64_t N, int32_t H, int32_t dk, int32_t dv,
 #pragma omp parallel
   {
     double* u = (double*)malloc(sizeof(double) * (size_t)dv);
-    if (!u) {
+    double* qkg = (double*)malloc(sizeof(double) * 3 * (size_t)dk);
+    if (!u || !qkg) {
 #pragma omp atomic write
       bad = 1;
     }
 #pragma omp for schedule(static)
     for (int64_t unit = 0; unit < N * (int64_t)H; ++unit) {
-      if (!u) continue;
+      if (!u || !qkg) continue;
       const int64_t n = unit / H;
       const int32_t h = (int32_t)(unit % H);
       const int64_t slot = state_indices ? state_indices[n] : n;
       double* S = state + ((size_t)slot * H + h) * state_elems;
       const size_t row = (size_t)unit; /* [N, H] row of the token inputs */
       double* o = out + row * dv;
-      token_step(dk, dv, S, q + row * dk, k + row * dk, v + row * dv,
-                 g + row * dk, (double)beta[row], scale, mode, u, o);
+      const double b = prep_token(dk, q + row * dk, k + row * dk, g + row * dk, beta[row],
+                                  mode, qkg, qkg + dk, qkg + 2 * dk);
+      token_step(dk, dv, S, qkg, qkg + dk, v + row * dv, qkg + 2 * dk, b, scale, mode, u, o);
       if (gate) rmsnorm_gate(dv, o, gate + row * dv, norm_weight, eps);
     }
     free(u);
+    free(qkg);
   }
   return bad ? KDA_REF_BAD_ARG : KDA_REF_OK;
 }

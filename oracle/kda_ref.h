@@ -46,8 +46,14 @@
 extern "C" {
 #endif
 
-/* mode bits (test-only variants of the recurrence) */
-#define KDA_REF_ERASE_OFF 1u /* drop the "- S^T k" term: u = beta v (gated linear attention) */
+/* mode bits */
+#define KDA_REF_ERASE_OFF 1u /* test-only: drop the "- S^T k" term: u = beta v (gated linear attention) */
+/* pre-processing of the raw projections (see prep_token in kda_ref.c) */
+#define KDA_REF_G_LOGITS 2u    /* g holds decay logits a: g = KDA_REF_G_MIN * sigmoid(a) */
+#define KDA_REF_BETA_LOGITS 4u /* beta holds logits b: beta = sigmoid(b) */
+#define KDA_REF_QK_L2NORM 8u   /* q, k <- x / sqrt(sum x^2 + KDA_REF_L2NORM_EPS) per (token, head) */
+#define KDA_REF_G_MIN (-5.0)
+#define KDA_REF_L2NORM_EPS 1e-6
 
 /* Return codes */
 #define KDA_REF_OK 0

@@ -176,6 +176,76 @@ def pin_snapshots_are_unrolled_prefix_states(ref, seed=7):
     assert row == snaps.shape[0]
 
 
+# --- pre-processing of the raw projections (decay logits, beta logits, q/k L2 norm) ----------
+def _small(seed, T=40, H=2, dk=8, dv=5):
+    rng = _rng(seed)
+    q = rng.standard_normal((T, H, dk)).astype(np.float32)
+    k = rng.standard_normal((T, H, dk)).astype(np.float32)
+    v = rng.standard_normal((T, H, dv)).astype(np.float32)
+    g = (-rng.random((T, H, dk))).astype(np.float32)
+    beta = rng.random((T, H)).astype(np.float32)
+    gate = rng.standard_normal((T, H, dv)).astype(np.float32)
+    s0 = rng.standard_normal((1, H, dk, dv))
+    return q, k, v, g, beta, gate, s0
+
+
+def pin_decay_logits_are_the_scaled_sigmoid(ref):
+    """g = -5 sigmoid(a): a = 0 gives g = -2.5 exactly, a = +40 the floor -5, a = -40 no decay
+    (sigmoid(-40) = 4e-18), each against a run given that g directly."""
+    q, k, v, g, beta, gate, s0 = _small(11)
+    for a_val, g_val, tol in ((0.0, -2.5, 1e-13), (40.0, -5.0, 1e-12), (-40.0, 0.0, 1e-12)):
+        a = np.full_like(g, a_val)
+        o1, f1 = ref.forward(q, k, v, a, beta, gate=gate, initial_state=s0, mode=ref.G_LOGITS)
+        o2, f2 = ref.forward(q, k, v, np.full_like(g, g_val), beta, gate=gate, initial_state=s0)
+        np.testing.assert_allclose(o1, o2, rtol=tol, atol=tol)
+        np.testing.assert_allclose(f1, f2, rtol=tol, atol=tol)
+
+
+def pin_beta_logits_are_the_sigmoid(ref):
+    """beta = sigmoid(b): b = 0 gives beta = 1/2 exactly; b = -40 removes the write (the pure
+    decay closed form of S0); b = +40 gives beta = 1."""
+    q, k, v, g, beta, gate, s0 = _small(12)
+    o1, f1 = ref.forward(q, k, v, g, np.zeros_like(beta), gate=gate, initial_state=s0, mode=ref.BETA_LOGITS)
+    o2, f2 = ref.forward(q, k, v, g, np.full_like(beta, 0.5), gate=gate, initial_state=s0)
+    np.testing.assert_allclose(o1, o2, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(f1, f2, rtol=1e-13, atol=1e-13)
+    o1, f1 = ref.forward(q, k, v, g, np.full_like(beta, 40.0), initial_state=s0, mode=ref.BETA_LOGITS)
+    o2, f2 = ref.forward(q, k, v, g, np.ones_like(beta), initial_state=s0)
+    np.testing.assert_allclose(f1, f2, rtol=1e-12, atol=1e-12)
+    _, f1 = ref.forward(q, k, v, g, np.full_like(beta, -40.0), initial_state=s0, mode=ref.BETA_LOGITS)
+    decay = np.exp(g.astype(np.float64).sum(axis=0))  # [H, dk]
+    np.testing.assert_allclose(f1[0], decay[:, :, None] * s0[0], rtol=1e-12, atol=1e-14)
+
+
+def pin_qk_l2norm_gives_unit_keys(ref):
+    """q, k <- x / sqrt(|x|^2 + 1e-6): (a) with beta = 1, g = 0 and keys of norm 3 the delta write
+    is the exact Householder projection of the normalised key, S_t^T k_t/|k_t| = v_t (to the
+    1e-7 the eps leaves); (b) scaling q by 4 and k by 1/4 changes nothing (to that eps)."""
+    rng = _rng(13)
+    T, dk, dv = 12, 16, 6
+    k = _exact_unit_rows(rng, T, dk)[:, None, :] * 3.0
+    q = rng.standard_normal((T, 1, dk)).astype(np.float32)
+    v = rng.standard_normal((T, 1, dv)).astype(np.float32)
+    g = np.zeros((T, 1, dk), np.float32)
+    s0 = rng.standard_normal((1, 1, dk, dv))
+    S = s0[0, 0].copy()
+    for t in range(T):
+        _, fin = ref.forward(q[:t + 1], k[:t + 1], v[:t + 1], g[:t + 1], np.ones((t + 1, 1), np.float32),
+                             initial_state=s0, mode=ref.QK_L2NORM)
+        kt = k[t, 0].astype(np.float64) / 3.0
+        np.testing.assert_allclose(fin[0, 0].T @ kt, v[t, 0], rtol=0, atol=2e-6)
+    q, k2, v, g, beta, gate, s0 = _small(14)
+    o1, f1 = ref.forward(q, k2, v, g, beta, gate=gate, initial_state=s0, mode=ref.QK_L2NORM)
+    o2, f2 = ref.forward(q * 4, k2 * 0.25, v, g, beta, gate=gate, initial_state=s0, mode=ref.QK_L2NORM)
+    # (the 1e-6 inside the root moves the scaled keys' norm by ~1e-6 relative; the RMSNorm
+    # epilogue can amplify that on small outputs)
+    np.testing.assert_allclose(o1, o2, rtol=2e-4, atol=2e-5)
+    np.testing.assert_allclose(f1, f2, rtol=2e-4, atol=2e-5)
+    # and the normalisation does act: the unnormalised run differs at order 1
+    o3, _ = ref.forward(q * 4, k2 * 0.25, v, g, beta, gate=gate, initial_state=s0)
+    assert np.abs(o3 - o1).max() > 1e-2
+
+
 # --- I4: orthonormal keys form an exact associative memory ----------------------------------
 def pin_orthonormal_keys_are_recalled_exactly(ref):
     """g = 0, beta = 1, keys = distinct rows of a normalised 16x16 Hadamard matrix (exactly
@@ -319,7 +389,8 @@ PINS = [pin_delta_write_is_exact_for_unit_keys, pin_beta_zero_is_pure_decay,
         pin_orthonormal_keys_are_recalled_exactly, pin_linear_in_values_and_initial_state,
         pin_split_invariance_and_varlen_packing, pin_epilogue_matches_library_rmsnorm,
         pin_decode_step_matches_one_token_forward, pin_scalar_worked_example,
-        pin_snapshots_are_unrolled_prefix_states]
+        pin_snapshots_are_unrolled_prefix_states, pin_decay_logits_are_the_scaled_sigmoid,
+        pin_beta_logits_are_the_sigmoid, pin_qk_l2norm_gives_unit_keys]
 
 
 @pytest.fixture(scope="module")

@@ -32,6 +32,10 @@ MUTANTS = [
     ("snapshot_wrong_head", "memcpy(snapshots + ((size_t)srow * H + h) * state_elems, S,",
      "memcpy(snapshots + ((size_t)srow * H + 0) * state_elems, S,"),
     ("snapshot_one_token_early", None, None),  # built below: the copy moved before the token's update
+    ("decay_logit_sign", "KDA_REF_G_MIN * sigmoid((double)g[i])", "KDA_REF_G_MIN * sigmoid(-(double)g[i])"),
+    ("beta_logit_ignored", "sigmoid((double)beta) : (double)beta", "(double)beta : (double)beta"),
+    ("l2norm_q_only", "kd[i] *= rk;", "kd[i] *= 1.0;"),
+    ("l2norm_eps_outside", "1.0 / sqrt(sk + KDA_REF_L2NORM_EPS)", "1.0 / (sqrt(sk) + 0.3)"),
 ]
 
 
@@ -62,7 +66,7 @@ def _mutant_source(name, old, new):
                       "sizeof(double) * state_elems);\n        }\n")
         snap = src[i:j]
         src = src[:i] + src[j:]
-        k = src.index("        token_step(dk, dv, S, q + row * dk, k + row * dk, v + row * dv,")
+        k = src.index("        const double b = prep_token(dk, q + row * dk, k + row * dk, g + row * dk, beta[row],")
         return src[:k] + snap + src[k:]
     assert old in src, f"mutation anchor for {name} not found"
     return src.replace(old, new, 1)
