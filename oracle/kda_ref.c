@@ -83,7 +83,7 @@ static void token_step(int32_t dk, int32_t dv, double* S, const double* q,
  *   KDA_REF_BETA_LOGITS: beta = sigmoid(b)
  *   KDA_REF_QK_L2NORM:   q <- q / sqrt(sum_i q_i^2 + 1e-6), the same for k
  *                        (unit-norm keys are what makes the delta write a
- *                        Householder projection: "Kimi K3 de Moonshot AI",
+ *                        Householder projection: "Kimi K3 from Moonshot AI",
  *                        section "Kimi Delta Attention (KDA)") */
 static double prep_token(int32_t dk, const float* q, const float* k, const float* g,
                          float beta, uint32_t mode, double* qd, double* kd, double* gd) {
