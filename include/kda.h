@@ -38,7 +38,8 @@
  *   - Precondition: every g lies in [KDA_G_MIN, 0].  Without KDA_FLAG_CHECK_DECAY a
  *     value below KDA_G_MIN is undefined behaviour for the bf16 tensor-core path
  *     (its tile factors may overflow); with the flag the kernel reports
- *     KDA_ERR_DECAY_OUT_OF_RANGE in the error word.
+ *     KDA_ERR_DECAY_OUT_OF_RANGE in the error word.  With KDA_FLAG_G_LOGITS the kernels
+ *     compute g = KDA_G_MIN * sigmoid(a) themselves and the bound holds by construction.
  *   - Outputs must not alias inputs.  Decode updates `state` in place by design.
  */
 #ifndef KDA_H
@@ -77,6 +78,17 @@ typedef enum kda_dtype {
 #define KDA_FLAG_CHECK_DECAY 0x1u      /* verify g in [KDA_G_MIN, 0] (and state indices) on the device */
 #define KDA_FLAG_FORCE_SIMT 0x2u       /* prefill: use the fp32 CUDA-core chunk kernel even for bf16 */
 #define KDA_FLAG_TEST_FORCE_TIMEOUT 0x4u /* tests only: bounded waits give up at once -> KDA_ERR_TIMEOUT */
+/* Pre-processing of the raw projections inside the kernels (prefill and decode), so that no
+ * separate pass reads and writes q, k, g and beta.  g_min = KDA_G_MIN: the scaled-sigmoid decay
+ * bound ("Kimi K3: Engineering a 2.8 Trillion Parameter Frontier", section "Dimension 1"; "Kimi
+ * K3 Architecture Explained", section "Token mixing"), which then holds by construction.  The L2
+ * norm makes the keys unit vectors, which the delta rule's Householder form assumes ("Kimi K3
+ * from Moonshot AI", section "Kimi Delta Attention (KDA)"); the pages do not give its epsilon:
+ * x / sqrt(sum x^2 + 1e-6) is taken here. */
+#define KDA_FLAG_G_LOGITS 0x8u     /* g holds decay logits a: the kernels use g = KDA_G_MIN * sigmoid(a) */
+#define KDA_FLAG_BETA_LOGITS 0x10u /* beta holds logits b: the kernels use sigmoid(b) */
+#define KDA_FLAG_QK_L2NORM 0x20u   /* q, k L2-normalised per (token, head): x / sqrt(sum_i x_i^2 + 1e-6) */
+#define KDA_L2NORM_EPS 1e-6f
 
 /* ------------------------------------------------------------------------------------------
  * Chunkwise prefill.

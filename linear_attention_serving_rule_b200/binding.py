@@ -34,6 +34,9 @@ KDA_F32 = 1
 KDA_FLAG_CHECK_DECAY = 0x1
 KDA_FLAG_FORCE_SIMT = 0x2
 KDA_FLAG_TEST_FORCE_TIMEOUT = 0x4
+KDA_FLAG_G_LOGITS = 0x8       # g holds decay logits a: the kernels use g = -5 sigmoid(a)
+KDA_FLAG_BETA_LOGITS = 0x10   # beta holds logits: the kernels use sigmoid(beta)
+KDA_FLAG_QK_L2NORM = 0x20     # q, k L2-normalised per (token, head) in the kernels
 
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
             "kda_read_device_error", "kda_status_string", "kda_chunk_fwd_noalloc",

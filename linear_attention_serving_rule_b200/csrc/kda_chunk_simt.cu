@@ -63,6 +63,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Seg seg = plan.seg[blockIdx.x / H];
   const int h = blockIdx.x % H;
   const bool checked = (p.flags & KDA_FLAG_CHECK_DECAY) != 0;
+  const bool g_logits = (p.flags & KDA_FLAG_G_LOGITS) != 0;
+  const bool b_logits = (p.flags & KDA_FLAG_BETA_LOGITS) != 0;
+  const bool l2norm = (p.flags & KDA_FLAG_QK_L2NORM) != 0;
   const bool write_out = (seg.role == kRoleWhole || seg.role == kRoleFromWs);
 
   // ---- start state
@@ -98,6 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (t < L) {
         const size_t r = ((size_t)(seg.tok0 + c0 + t) * H + h) * DK + c;
         qx = to_f32(q[r]); kx = to_f32(k[r]); gx = to_f32(g[r]);
+        if (g_logits) gx = KDA_G_MIN / (1.f + expf(-gx));  // g = g_min sigmoid(a)
         if (checked && !(gx >= KDA_G_MIN && gx <= 0.f)) report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
       }
       sm.Qt[idx] = qx; sm.Kt[idx] = kx; sm.G[idx] = gx;
@@ -106,8 +110,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = idx / DV, j = idx - t * DV;
       sm.V[idx] = (t < L) ? to_f32(v[((size_t)(seg.tok0 + c0 + t) * H + h) * DV + j]) : 0.f;
     }
-    if (tid < kC) sm.beta[tid] = (tid < L) ? to_f32(bt[(size_t)(seg.tok0 + c0 + tid) * H + h]) : 0.f;
+    if (tid < kC) {
+      float b = (tid < L) ? to_f32(bt[(size_t)(seg.tok0 + c0 + tid) * H + h]) : 0.f;
+      if (b_logits && tid < L) b = 1.f / (1.f + expf(-b));  // beta = sigmoid(b)
+      sm.beta[tid] = b;
+    }
     __syncthreads();
+    if (l2norm) {  // q, k <- x / sqrt(|x|^2 + eps), one warp per row (padding rows stay zero)
+      const int wq = tid >> 5, lq = tid & 31;
+      for (int r = wq; r < 2 * kC; r += kThreads / 32) {
+        float* xr = (r < kC ? sm.Qt : sm.Kt) + (r % kC) * DK;
+        float ss = 0.f;
+        for (int c = lq; c < DK; c += 32) ss += xr[c] * xr[c];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float rn = rsqrtf(ss + KDA_L2NORM_EPS);
+        for (int c = lq; c < DK; c += 32) xr[c] *= rn;
+      }
+      __syncthreads();
+    }
     // ---- decay factors: one thread per key channel scans the chunk
     if (tid < DK) {
       const int c = tid;

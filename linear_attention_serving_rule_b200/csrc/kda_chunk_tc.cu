@@ -93,6 +93,7 @@ struct Misc {
   float ec[DK];     // e^{gamma_C}
   float nw[DV];     // RMSNorm weight (1 without one)
   float ssq[2][C];  // epilogue: per-row sums of squares of the two column halves
+  float qkss[2][2 * C];  // with KDA_FLAG_QK_L2NORM: sums of squares of the k|q rows, by column half
 };
 static_assert(sizeof(Misc) <= 8192, "misc block too large");
 
@@ -197,6 +198,9 @@ __device__ __forceinline__ void umma_k_loop(uint32_t d, uint32_t a_addr, uint32_
   }
 }
 
+// kPre: the decay-logit and q/k L2-norm pre-processing (KDA_FLAG_G_LOGITS, KDA_FLAG_QK_L2NORM) is
+// compiled in; the instance without it keeps the plain path free of their branches.
+template <bool kPre>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ Plan plan, const __grid_constant__ TcMaps maps, const ChunkParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -213,6 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int h = blockIdx.x % H;
   const bool has_gate = p.gate != nullptr;
   const bool checked = (p.flags & KDA_FLAG_CHECK_DECAY) != 0;
+  const bool g_logits = kPre && (p.flags & KDA_FLAG_G_LOGITS) != 0;
+  const bool l2norm = kPre && (p.flags & KDA_FLAG_QK_L2NORM) != 0;
   const uint64_t limit = (p.flags & KDA_FLAG_TEST_FORCE_TIMEOUT) ? 0ull : 2000000000ull;  // 2 s
   const uint64_t drain_limit = 2000000000ull;
   const int nchunks = (seg.len + C - 1) / C;
@@ -254,7 +260,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int t = lane + 32 * r;
-        m->beta[j & 1][t] = (t < L) ? to_f32(static_cast<const __nv_bfloat16*>(p.beta)[(size_t)(tok + t) * H + h]) : 0.f;
+        float bv = (t < L) ? to_f32(static_cast<const __nv_bfloat16*>(p.beta)[(size_t)(tok + t) * H + h]) : 0.f;
+        if ((p.flags & KDA_FLAG_BETA_LOGITS) && t < L) bv = 1.f / (1.f + expf(-bv));  // beta = sigmoid(b)
+        m->beta[j & 1][t] = bv;
       }
       __syncwarp();
       if (lane == 0) {
@@ -471,6 +479,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 8; ++e) g8[e] = 0.f;
         }
+        if (g_logits && t < L) {  // g = g_min sigmoid(a); the exponent is clamped to keep 1 + e finite
+#pragma unroll
+          for (int e = 0; e < 8; ++e) g8[e] = __fdividef(KDA_G_MIN, 1.f + ex2(fminf(-g8[e] * kLog2e, 126.f)));
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           bad |= !(g8[e] >= KDA_G_MIN && g8[e] <= 0.f);
@@ -513,6 +525,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------------- decay prep: all bf16 operands
 
       if (!wg_wait(&m->full_kq, par)) { ok = false; break; }
+      if (l2norm) {  // sums of squares of the raw k | q rows (two column halves per row)
+        const int rr = tid & 127, hf = tid >> 7;
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          float f[8];
+          unpack8(at16(sm, OFF_KQ + sw128_oct(rr, 8 * hf + i, 16384)), f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ss += f[e] * f[e];
+        }
+        m->qkss[hf][rr] = ss;
+        sync_wg();
+      }
       // Per-channel factors, applied so that no O(1) value is multiplied by an underflowed
       // constant: with se_m = e^{decay over sub-tile m}, Eb = e^{r_b} = prod_{m<b} se_m, and per
       // token ix = e^{r_b - gamma_t} in [1, e^80]; the chain ix, ix se_b, ix se_b se_{b+1}, ...
@@ -542,6 +567,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (t < L) {
             unpack8(at16(sm, OFF_KQ + sw128_oct(t, o, 16384)), kf);
             unpack8(at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)), qf);
+            if (l2norm) {  // x / sqrt(|x|^2 + eps)
+              const float rk = rsqrtf(m->qkss[0][t] + m->qkss[1][t] + KDA_L2NORM_EPS);
+              const float rq = rsqrtf(m->qkss[0][64 + t] + m->qkss[1][64 + t] + KDA_L2NORM_EPS);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) { kf[e] *= rk; qf[e] *= rq; }
+            }
           } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e) { kf[e] = 0.f; qf[e] = 0.f; }
@@ -978,9 +1009,11 @@ cudaError_t launch_chunk_tc(const Plan& plan, const ChunkParams& p, cudaStream_t
   if (!make_map(&maps.q, p.q, p.H, T) || !make_map(&maps.k, p.k, p.H, T) || !make_map(&maps.g, p.g, p.H, T) ||
       !make_map(&maps.v, p.v, p.H, T))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  const bool pre = (p.flags & (KDA_FLAG_G_LOGITS | KDA_FLAG_QK_L2NORM)) != 0;
+  auto kern = pre ? chunk_tc_kernel<true> : chunk_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  chunk_tc_kernel<<<plan.n_seg * plan.H, kThreads, SMEM_BYTES, stream>>>(plan, maps, p);
+  kern<<<plan.n_seg * plan.H, kThreads, SMEM_BYTES, stream>>>(plan, maps, p);
   return cudaGetLastError();
 }
 

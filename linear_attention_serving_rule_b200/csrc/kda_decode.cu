@@ -40,7 +40,9 @@ struct DecodeParams {
   uint32_t* error_word;
 };
 
-template <typename T, int DK, int DV>
+// kPre: the pre-processing of the raw projections (KDA_FLAG_G_LOGITS, KDA_FLAG_BETA_LOGITS,
+// KDA_FLAG_QK_L2NORM) is compiled in; the instance without it is the plain step.
+template <typename T, int DK, int DV, bool kPre>
 __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams p) {
   constexpr int TPR = DV / 4;              // threads per state row (one float4 each)
   constexpr int RPP = kThreads / TPR;      // rows per pass
@@ -52,7 +54,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   __shared__ float so[DV];
   __shared__ __align__(16) float red_k[RPP][DV];
   __shared__ __align__(16) float red_q[RPP][DV];
-  __shared__ float s_kq;
+  __shared__ float s_kq, s_rk, s_rq;  // k.q of the normalised vectors; 1/|k|, 1/|q| (or 1)
   __shared__ float s_ss[DV / 32 > 0 ? DV / 32 : 1];
 
   const int tid = threadIdx.x;
@@ -60,6 +62,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   const int n = unit / p.H;
   const int h = unit - n * p.H;
   const bool checked = (p.flags & KDA_FLAG_CHECK_DECAY) != 0;
+  const bool g_logits = kPre && (p.flags & KDA_FLAG_G_LOGITS) != 0;
+  const bool l2norm = kPre && (p.flags & KDA_FLAG_QK_L2NORM) != 0;
 
   int slot = p.state_indices ? p.state_indices[n] : n;
   if (slot < 0 || slot >= p.num_slots) {  // uniform over the block
@@ -82,17 +86,38 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   for (int i = tid; i < DK; i += kThreads) {
     sk[i] = to_f32(kp[i]);
     sq[i] = to_f32(qp[i]);
-    const float gi = to_f32(gp[i]);
+    float gi = to_f32(gp[i]);
+    if (g_logits) gi = KDA_G_MIN / (1.f + expf(-gi));  // g = g_min sigmoid(a)
     if (checked && !(gi >= KDA_G_MIN && gi <= 0.0f)) report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
     sa[i] = expf(gi);
   }
   __syncthreads();
+  // With KDA_FLAG_QK_L2NORM the state pass below runs on the raw k and q: S'^T k and S'^T q are
+  // linear in them, so 1/|k| and 1/|q| are applied to the reductions and to the write instead.
   if (tid < 32) {
-    float acc = 0.f;
-    for (int i = tid; i < DK; i += 32) acc += sk[i] * sq[i];
+    float acc = 0.f, kk = 0.f, qq = 0.f;
+    for (int i = tid; i < DK; i += 32) {
+      acc += sk[i] * sq[i];
+      if (kPre) {
+        kk += sk[i] * sk[i];
+        qq += sq[i] * sq[i];
+      }
+    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (tid == 0) s_kq = acc;
+    for (int o = 16; o > 0; o >>= 1) {
+      acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (kPre) {
+        kk += __shfl_xor_sync(0xffffffffu, kk, o);
+        qq += __shfl_xor_sync(0xffffffffu, qq, o);
+      }
+    }
+    if (tid == 0) {
+      const float rk = l2norm ? rsqrtf(kk + KDA_L2NORM_EPS) : 1.f;
+      const float rq = l2norm ? rsqrtf(qq + KDA_L2NORM_EPS) : 1.f;
+      s_rk = rk;
+      s_rq = rq;
+      s_kq = acc * rk * rq;
+    }
   }
 
   float4 yk = make_float4(0.f, 0.f, 0.f, 0.f), yq = yk;
@@ -108,15 +133,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   reinterpret_cast<float4*>(red_q[r0])[cg] = yq;
   __syncthreads();
 
-  const float beta = to_f32(static_cast<const T*>(p.beta)[row]);
+  float beta = to_f32(static_cast<const T*>(p.beta)[row]);
+  if (kPre && (p.flags & KDA_FLAG_BETA_LOGITS)) beta = 1.f / (1.f + expf(-beta));  // beta = sigmoid(b)
+  const float rk = kPre ? s_rk : 1.f;
   if (tid < DV) {
     float ak = 0.f, aq = 0.f;
 #pragma unroll
     for (int r = 0; r < RPP; ++r) { ak += red_k[r][tid]; aq += red_q[r][tid]; }
     const float vj = to_f32(static_cast<const T*>(p.v)[row * DV + tid]);
-    const float u = beta * (vj - ak);
+    const float u = beta * (vj - ak * rk);
     su[tid] = u;
-    so[tid] = p.scale * (aq + u * s_kq);
+    so[tid] = p.scale * (kPre ? aq * s_rq + u * s_kq : aq + u * s_kq);
   }
   __syncthreads();
 
@@ -124,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
 #pragma unroll
   for (int i = 0; i < NP; ++i) {
     const int r = r0 + RPP * i;
-    const float kr = sk[r];
+    const float kr = sk[r] * rk;
     s[i].x += kr * u4.x; s[i].y += kr * u4.y; s[i].z += kr * u4.z; s[i].w += kr * u4.w;
     __stcs(reinterpret_cast<float4*>(S + (size_t)r * DV) + cg, s[i]);
   }
@@ -158,7 +185,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
 
 template <typename T, int DK, int DV>
 cudaError_t launch_t(const DecodeParams& p, int units, cudaStream_t stream) {
-  decode_kernel<T, DK, DV><<<units, kThreads, 0, stream>>>(p);
+  if (p.flags & (KDA_FLAG_G_LOGITS | KDA_FLAG_BETA_LOGITS | KDA_FLAG_QK_L2NORM))
+    decode_kernel<T, DK, DV, true><<<units, kThreads, 0, stream>>>(p);
+  else
+    decode_kernel<T, DK, DV, false><<<units, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -95,9 +95,13 @@ def _randn(shape, gen, device):
 def make_prefill(*, H: int, dk: int, dv: int, dtype="bf16", seed: int = 0,
                  device="cpu", lengths=None, B: int | None = None, T: int | None = None,
                  gate: bool = True, init_state: bool = False, decay_shift: float = 0.0,
-                 state_std: float = 0.02) -> PrefillInputs:
+                 state_std: float = 0.02, raw: bool = False) -> PrefillInputs:
     """Packed prefill inputs.  Give either `lengths` (varlen) or B and T (B equal
-    sequences of T tokens, stored packed as [B*T, H, d])."""
+    sequences of T tokens, stored packed as [B*T, H, d]).
+
+    raw=True returns the same draws before their last step: q and k not L2-normalised, beta
+    and g as the logits b and a of beta = sigmoid(b), g = -5 sigmoid(a) (the inputs of the
+    library's pre-processing flags)."""
     if lengths is None:
         lengths = np.full(B, T, dtype=np.int64)
     cu = cu_from_lengths(lengths)
@@ -106,11 +110,14 @@ def make_prefill(*, H: int, dk: int, dv: int, dtype="bf16", seed: int = 0,
     dt = torch_dtype(dtype)
     gen = torch.Generator(device=device)
     gen.manual_seed(int(seed))
-    q = _l2norm(_randn((T_tot, H, dk), gen, device)).to(dt)
-    k = _l2norm(_randn((T_tot, H, dk), gen, device)).to(dt)
+    nrm = (lambda x: x) if raw else _l2norm
+    q = nrm(_randn((T_tot, H, dk), gen, device)).to(dt)
+    k = nrm(_randn((T_tot, H, dk), gen, device)).to(dt)
     v = _randn((T_tot, H, dv), gen, device).to(dt)
-    beta = torch.sigmoid(_randn((T_tot, H), gen, device)).to(dt)
-    g = (G_MIN * torch.sigmoid(_randn((T_tot, H, dk), gen, device) + decay_shift)).to(dt)
+    b_logit = _randn((T_tot, H), gen, device)
+    beta = (b_logit if raw else torch.sigmoid(b_logit)).to(dt)
+    a_logit = _randn((T_tot, H, dk), gen, device) + decay_shift
+    g = (a_logit if raw else G_MIN * torch.sigmoid(a_logit)).to(dt)
     gt = _randn((T_tot, H, dv), gen, device).to(dt) if gate else None
     s0 = (state_std * _randn((N, H, dk, dv), gen, device)) if init_state else None
     return PrefillInputs(q, k, v, g, beta, gt, s0, cu)
@@ -126,7 +133,7 @@ def make_workload(name: str, device="cpu", **overrides) -> PrefillInputs:
     return make_prefill(H=w["H"], dk=w["dk"], dv=w["dv"], dtype=w["dtype"], seed=w["seed"],
                         device=device, lengths=lengths, B=w.get("B"), T=w.get("T"),
                         gate=w["gate"], init_state=w["init_state"],
-                        decay_shift=w.get("decay_shift", 0.0))
+                        decay_shift=w.get("decay_shift", 0.0), raw=w.get("raw", False))
 
 
 @dataclass
@@ -140,10 +147,11 @@ class DecodeInputs:
 
 
 def make_decode_token(*, N: int, H: int, dk: int, dv: int, dtype="bf16", seed: int = 0,
-                      device="cpu", gate: bool = True, decay_shift: float = 0.0) -> DecodeInputs:
+                      device="cpu", gate: bool = True, decay_shift: float = 0.0,
+                      raw: bool = False) -> DecodeInputs:
     """Inputs of one decode step (one token per sequence)."""
     p = make_prefill(H=H, dk=dk, dv=dv, dtype=dtype, seed=seed, device=device,
-                     lengths=np.ones(N, dtype=np.int64), gate=gate, decay_shift=decay_shift)
+                     lengths=np.ones(N, dtype=np.int64), gate=gate, decay_shift=decay_shift, raw=raw)
     return DecodeInputs(p.q, p.k, p.v, p.g, p.beta, p.gate)
 
 

@@ -24,16 +24,16 @@ def host(t):
     return None if t is None else t.detach().float().cpu().numpy()
 
 
-def oracle_full(inp, norm_weight=None, eps=1e-6, num_threads=0):
+def oracle_full(inp, norm_weight=None, eps=1e-6, num_threads=0, mode=0):
     """The oracle on every unit of a (small) packed PrefillInputs."""
     a = {n: host(getattr(inp, n)) for n in ("q", "k", "v", "g", "beta", "gate")}
     s0 = None if inp.initial_state is None else inp.initial_state.double().cpu().numpy()
     return oracle.forward(a["q"], a["k"], a["v"], a["g"], a["beta"], cu_seqlens=inp.cu_seqlens,
                           gate=a["gate"], initial_state=s0, norm_weight=host(norm_weight), eps=eps,
-                          num_threads=num_threads)
+                          num_threads=num_threads, mode=mode)
 
 
-def oracle_units(inp, units, *, tok_limit=None, norm_weight=None, eps=1e-6, num_threads=0):
+def oracle_units(inp, units, *, tok_limit=None, norm_weight=None, eps=1e-6, num_threads=0, mode=0):
     """Oracle outputs and final states for the listed (n, h) units only.
 
     Returns {(n, h): (out [len, dv] float64, final [dk, dv] float64)}.  With tok_limit the
@@ -60,7 +60,8 @@ def oracle_units(inp, units, *, tok_limit=None, norm_weight=None, eps=1e-6, num_
     s0 = np.stack(s0s)[:, None] if s0s else None
     out, fin = oracle.forward(cat(qs), cat(ks), cat(vs), cat(gs), cat(bs), cu_seqlens=cuu,
                               gate=cat(gts) if gts else None, initial_state=s0,
-                              norm_weight=host(norm_weight), eps=eps, num_threads=num_threads)
+                              norm_weight=host(norm_weight), eps=eps, num_threads=num_threads,
+                              mode=mode)
     res = {}
     for i, u in enumerate(units):
         res[u] = (out[cuu[i]:cuu[i + 1], 0], fin[i, 0])
