@@ -350,8 +350,10 @@ def run_ours(args):
 
     # ---------------- decode workload
     decode = None
+    decode_multi = None
     if not args.no_decode:
         decode = run_decode(args, dev, stream, rank, world, peaks, peak_src, clocks)
+        decode_multi = run_decode_multi(args, dev, stream, rank, peaks, decode["roofline"]["kernel_ms"])
     clocks.stop()
     clk = clocks.summary()
 
@@ -380,7 +382,7 @@ def run_ours(args):
                        "l2": f"inputs {input_bytes / 2**20:.0f} MiB per step > 126 MiB L2; no flush"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_call * args.steps, "clocks": clk, "decode": decode,
-            "snapshots": snaps, "preprocess": prep}
+            "snapshots": snaps, "preprocess": prep, "decode_multi": decode_multi}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -565,6 +567,49 @@ def run_decode(args, dev, stream, rank, world, peaks, peak_src, clocks):
                          "alg_bytes_per_launch": state_bytes, "kernel_ms": kern_ms,
                          "kernel_source_sha1": sha},
             "gpu_launches": steps}
+
+
+def run_decode_multi(args, dev, stream, rank, peaks, single_ms, K=4):
+    """The decode batch verifying K draft tokens per sequence in one call (state read once and
+    written once): kernel time, tokens/s and state GB/s, and the per-token cost against K
+    single-token steps."""
+    import numpy as np
+    import torch
+    import linear_attention_serving_rule_b200 as kda
+    from linear_attention_serving_rule_b200 import synth
+    w = synth.WORKLOADS[DECODE]
+    N, H, dk, dv = w["N"], w["H"], w["dk"], w["dv"]
+    seed = rank_seed(w["seed"], rank) + 100
+    state = synth.make_states(slots=N, H=H, dk=dk, dv=dv, seed=seed, device=dev)
+    p = synth.make_prefill(H=H, dk=dk, dv=dv, dtype="bf16", seed=seed + 1, device=dev,
+                           lengths=np.full(N, K, dtype=np.int64), gate=True)
+    t = [getattr(p, n).reshape((N, K) + tuple(getattr(p, n).shape[1:])).contiguous()
+         for n in ("q", "k", "v", "g", "beta", "gate")]
+    out = torch.empty((N, K, H, dv), dtype=torch.bfloat16, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def call():
+        kda.kda_decode_step(*t[:5], state, gate=t[5], out=out, error_word=err, stream=stream)
+    for _ in range(5):
+        call()
+    n = 50
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    torch.cuda.synchronize(dev)
+    for i in range(n):
+        ev[i][0].record(stream)
+        call()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    st = kda.kda_read_device_error(err)
+    if st != 0:
+        raise RuntimeError(f"multi-token decode device error: {kda.kda_status_string(st)}")
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    state_bytes = 2 * N * H * dk * dv * 4
+    return {"workload": f"decode bf16 N{N} x H{H} dk=dv={dk}, K={K} tokens per sequence per call",
+            "tokens_per_call": K, "launches": n, "kernel_ms": ms, "tokens_per_s": N * K / (ms / 1e3),
+            "state_gbs": state_bytes / (ms / 1e3) / 1e9,
+            "state_frac_of_peak": state_bytes / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+            "ms_per_token_vs_single_step": ms / K / single_ms}
 
 
 def main():

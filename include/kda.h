@@ -89,6 +89,7 @@ typedef enum kda_dtype {
 #define KDA_FLAG_BETA_LOGITS 0x10u /* beta holds logits b: the kernels use sigmoid(b) */
 #define KDA_FLAG_QK_L2NORM 0x20u   /* q, k L2-normalised per (token, head): x / sqrt(sum_i x_i^2 + 1e-6) */
 #define KDA_L2NORM_EPS 1e-6f
+#define KDA_FLAG_DECODE_NO_COMMIT 0x40u /* decode: leave `state` unchanged (verify pass; see tokens) */
 
 /* ------------------------------------------------------------------------------------------
  * Chunkwise prefill.
@@ -165,16 +166,27 @@ kda_status kda_chunk_fwd_workspace_size(const kda_chunk_args* args, size_t* byte
 kda_status kda_chunk_fwd(const kda_chunk_args* args, void* cuda_stream);
 
 /* ------------------------------------------------------------------------------------------
- * Decode step: one new token for each of N sequences, states updated in place.
+ * Decode step: K = tokens new tokens (K = 1 by default) for each of N sequences, states
+ * updated in place.
  *
- *   q, k, g       [N, H, dk]  dtype;  v, gate [N, H, dv] dtype (gate NULL => no epilogue)
- *   beta          [N, H]      dtype
- *   state         [num_slots, H, dk, dv] float32, read and written in place
+ *   q, k, g       [N, K, H, dk]  dtype;  v, gate [N, K, H, dv] dtype (gate NULL => no epilogue)
+ *   beta          [N, K, H]      dtype
+ *   state         [num_slots, H, dk, dv] float32, read once and (unless
+ *                 KDA_FLAG_DECODE_NO_COMMIT) written once, after the K tokens
  *   state_indices [N] int32 device pointer (sequence n uses slot state_indices[n]) or NULL
  *                 (slot n; then num_slots >= N).  Slots used by two sequences race.
- *   out           [N, H, dv]  dtype
+ *   out           [N, K, H, dv]  dtype: the output of every position
+ *   tokens        K >= 1 (0 is taken as 1): the sequence's next K tokens, in order
+ *   position_states [N, K, H, dk, dv] float32 or NULL: the state after each position
  *   error_word    device uint32 or NULL.  Sticky: kernels only set it; the caller zeroes it
  *                 before first use and kda_read_device_error zeroes it after reading.
+ *
+ * K > 1 serves speculative decoding (the model's multi-token-prediction layer drafts tokens for
+ * EAGLE-3 verification: "Kimi K3: Engineering a 2.8 Trillion Parameter Frontier", section
+ * "Infrastructure: The Physics of Running a 3T Model"): one call
+ * verifies K draft tokens with the state read once.  To roll back to the first m accepted
+ * tokens, either keep the position states and take position m - 1 as the new state, or verify
+ * with KDA_FLAG_DECODE_NO_COMMIT and then commit with a second call on the m accepted tokens.
  * ------------------------------------------------------------------------------------------ */
 typedef struct kda_decode_args {
   int32_t N, H, dk, dv;
@@ -194,6 +206,8 @@ typedef struct kda_decode_args {
   float eps;
   uint32_t flags;
   uint32_t* error_word;
+  int32_t tokens;
+  float* position_states;
 } kda_decode_args;
 
 kda_status kda_decode_step(const kda_decode_args* args, void* cuda_stream);

@@ -37,6 +37,7 @@ KDA_FLAG_TEST_FORCE_TIMEOUT = 0x4
 KDA_FLAG_G_LOGITS = 0x8       # g holds decay logits a: the kernels use g = -5 sigmoid(a)
 KDA_FLAG_BETA_LOGITS = 0x10   # beta holds logits: the kernels use sigmoid(beta)
 KDA_FLAG_QK_L2NORM = 0x20     # q, k L2-normalised per (token, head) in the kernels
+KDA_FLAG_DECODE_NO_COMMIT = 0x40  # decode: leave the state unchanged (verify pass)
 
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
             "kda_read_device_error", "kda_status_string", "kda_chunk_fwd_noalloc",
@@ -69,7 +70,7 @@ class KdaDecodeArgs(ctypes.Structure):
         ("norm_weight", _P), ("state", _P), ("num_slots", ctypes.c_int32),
         ("state_indices", _P), ("out", _P),
         ("scale", ctypes.c_float), ("eps", ctypes.c_float), ("flags", ctypes.c_uint32),
-        ("error_word", _P),
+        ("error_word", _P), ("tokens", ctypes.c_int32), ("position_states", _P),
     ]
 
 
@@ -282,14 +283,20 @@ def kda_chunk_fwd_noalloc(q, k, v, g, beta, *, gate=None, cu_seqlens=None, initi
 
 
 def kda_decode_step(q, k, v, g, beta, state, *, gate=None, state_indices=None, norm_weight=None,
-                    out=None, scale=0.0, eps=1e-6, flags=0, error_word=None, stream=None):
-    """One decode token per sequence through the C ABI; `state` [slots, H, dk, dv] fp32 is
-    updated in place.  Returns out [N, H, dv]."""
-    _check_cuda(q, k, v, g, beta, state, gate, state_indices, norm_weight)
-    N, H, dk = q.shape
+                    out=None, scale=0.0, eps=1e-6, flags=0, error_word=None, stream=None,
+                    position_states=None):
+    """Decode through the C ABI; `state` [slots, H, dk, dv] fp32 is updated in place (unless
+    KDA_FLAG_DECODE_NO_COMMIT).  q [N, H, dk] is one token per sequence; q [N, K, H, dk] is the
+    next K tokens of each sequence, with outputs for every position and, if position_states
+    [N, K, H, dk, dv] fp32 is given, the state after each position.  Returns out."""
+    _check_cuda(q, k, v, g, beta, state, gate, state_indices, norm_weight, position_states)
+    if q.dim() == 4:
+        N, K, H, dk = q.shape
+    else:
+        (N, H, dk), K = q.shape, 1
     dv = v.shape[-1]
     if out is None:
-        out = torch.empty((N, H, dv), dtype=v.dtype, device=v.device)
+        out = torch.empty(tuple(q.shape[:-1]) + (dv,), dtype=v.dtype, device=v.device)
     a = KdaDecodeArgs()
     a.N, a.H, a.dk, a.dv = N, H, dk, dv
     a.dtype = _dtype_code(q)
@@ -300,6 +307,7 @@ def kda_decode_step(q, k, v, g, beta, state, *, gate=None, state_indices=None, n
     a.out = _ptr(out)
     a.scale, a.eps, a.flags = float(scale), float(eps), int(flags)
     a.error_word = _ptr(error_word)
+    a.tokens, a.position_states = K, _ptr(position_states)
     rc = lib().kda_decode_step(ctypes.byref(a), _stream(stream))
     if rc != KDA_OK:
         raise KdaError(rc, "kda_decode_step")

@@ -309,6 +309,9 @@ extern "C" kda_status kda_decode_step(const kda_decode_args* a, void* cuda_strea
   if ((a->dk != 64 && a->dk != 128) || (a->dv != 64 && a->dv != 128)) return KDA_ERR_UNSUPPORTED;
   if (!(a->eps >= 0.f) || !(a->scale >= 0.f)) return KDA_ERR_INVALID_ARGUMENT;
   if ((int64_t)a->N * a->H > INT32_MAX) return KDA_ERR_UNSUPPORTED;
+  if (a->tokens < 0) return KDA_ERR_INVALID_ARGUMENT;
+  if ((int64_t)a->N * (a->tokens > 0 ? a->tokens : 1) * a->H > INT32_MAX) return KDA_ERR_UNSUPPORTED;
+  if (a->position_states && !aligned16(a->position_states)) return KDA_ERR_INVALID_ARGUMENT;
   if (a->N > 0) {
     const void* req[] = {a->q, a->k, a->v, a->g, a->state, a->out};
     for (const void* p : req)

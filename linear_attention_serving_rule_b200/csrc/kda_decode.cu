@@ -34,7 +34,8 @@ struct DecodeParams {
   float* state;
   const int32_t* state_indices;
   void* out;
-  int32_t H, num_slots;
+  float* position_states;  // [N, K, H, dk, dv] or null
+  int32_t H, num_slots, tokens;
   float scale, eps;
   uint32_t flags;
   uint32_t* error_word;
@@ -79,107 +80,118 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   for (int i = 0; i < NP; ++i)
     s[i] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)(r0 + RPP * i) * DV) + cg);
 
-  const size_t row = (size_t)unit;  // token inputs are [N, H, d]
-  const T* kp = static_cast<const T*>(p.k) + row * DK;
-  const T* qp = static_cast<const T*>(p.q) + row * DK;
-  const T* gp = static_cast<const T*>(p.g) + row * DK;
-  for (int i = tid; i < DK; i += kThreads) {
-    sk[i] = to_f32(kp[i]);
-    sq[i] = to_f32(qp[i]);
-    float gi = to_f32(gp[i]);
-    if (g_logits) gi = KDA_G_MIN / (1.f + expf(-gi));  // g = g_min sigmoid(a)
-    if (checked && !(gi >= KDA_G_MIN && gi <= 0.0f)) report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
-    sa[i] = expf(gi);
-  }
-  __syncthreads();
-  // With KDA_FLAG_QK_L2NORM the state pass below runs on the raw k and q: S'^T k and S'^T q are
-  // linear in them, so 1/|k| and 1/|q| are applied to the reductions and to the write instead.
-  if (tid < 32) {
-    float acc = 0.f, kk = 0.f, qq = 0.f;
-    for (int i = tid; i < DK; i += 32) {
-      acc += sk[i] * sq[i];
-      if (kPre) {
-        kk += sk[i] * sk[i];
-        qq += sq[i] * sq[i];
+  const int K = p.tokens;
+  const bool commit = (p.flags & KDA_FLAG_DECODE_NO_COMMIT) == 0;
+  // K tokens of the sequence in order; the state stays in registers between them
+  for (int tk = 0; tk < K; ++tk) {
+    if (tk > 0) __syncthreads();  // the previous token's shared arrays are consumed
+    const size_t row = ((size_t)n * K + tk) * p.H + h;  // token inputs are [N, K, H, d]
+    const T* kp = static_cast<const T*>(p.k) + row * DK;
+    const T* qp = static_cast<const T*>(p.q) + row * DK;
+    const T* gp = static_cast<const T*>(p.g) + row * DK;
+    for (int i = tid; i < DK; i += kThreads) {
+      sk[i] = to_f32(kp[i]);
+      sq[i] = to_f32(qp[i]);
+      float gi = to_f32(gp[i]);
+      if (g_logits) gi = KDA_G_MIN / (1.f + expf(-gi));  // g = g_min sigmoid(a)
+      if (checked && !(gi >= KDA_G_MIN && gi <= 0.0f)) report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
+      sa[i] = expf(gi);
+    }
+    __syncthreads();
+    // With KDA_FLAG_QK_L2NORM the state pass below runs on the raw k and q: S'^T k and S'^T q are
+    // linear in them, so 1/|k| and 1/|q| are applied to the reductions and to the write instead.
+    if (tid < 32) {
+      float acc = 0.f, kk = 0.f, qq = 0.f;
+      for (int i = tid; i < DK; i += 32) {
+        acc += sk[i] * sq[i];
+        if (kPre) {
+          kk += sk[i] * sk[i];
+          qq += sq[i] * sq[i];
+        }
+      }
+  #pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (kPre) {
+          kk += __shfl_xor_sync(0xffffffffu, kk, o);
+          qq += __shfl_xor_sync(0xffffffffu, qq, o);
+        }
+      }
+      if (tid == 0) {
+        const float rk = l2norm ? rsqrtf(kk + KDA_L2NORM_EPS) : 1.f;
+        const float rq = l2norm ? rsqrtf(qq + KDA_L2NORM_EPS) : 1.f;
+        s_rk = rk;
+        s_rq = rq;
+        s_kq = acc * rk * rq;
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (kPre) {
-        kk += __shfl_xor_sync(0xffffffffu, kk, o);
-        qq += __shfl_xor_sync(0xffffffffu, qq, o);
-      }
+
+    float4 yk = make_float4(0.f, 0.f, 0.f, 0.f), yq = yk;
+  #pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      const int r = r0 + RPP * i;
+      const float a = sa[r], kr = sk[r], qr = sq[r];
+      s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
+      yk.x += s[i].x * kr; yk.y += s[i].y * kr; yk.z += s[i].z * kr; yk.w += s[i].w * kr;
+      yq.x += s[i].x * qr; yq.y += s[i].y * qr; yq.z += s[i].z * qr; yq.w += s[i].w * qr;
     }
-    if (tid == 0) {
-      const float rk = l2norm ? rsqrtf(kk + KDA_L2NORM_EPS) : 1.f;
-      const float rq = l2norm ? rsqrtf(qq + KDA_L2NORM_EPS) : 1.f;
-      s_rk = rk;
-      s_rq = rq;
-      s_kq = acc * rk * rq;
+    reinterpret_cast<float4*>(red_k[r0])[cg] = yk;
+    reinterpret_cast<float4*>(red_q[r0])[cg] = yq;
+    __syncthreads();
+
+    float beta = to_f32(static_cast<const T*>(p.beta)[row]);
+    if (kPre && (p.flags & KDA_FLAG_BETA_LOGITS)) beta = 1.f / (1.f + expf(-beta));  // beta = sigmoid(b)
+    const float rk = kPre ? s_rk : 1.f;
+    if (tid < DV) {
+      float ak = 0.f, aq = 0.f;
+  #pragma unroll
+      for (int r = 0; r < RPP; ++r) { ak += red_k[r][tid]; aq += red_q[r][tid]; }
+      const float vj = to_f32(static_cast<const T*>(p.v)[row * DV + tid]);
+      const float u = beta * (vj - ak * rk);
+      su[tid] = u;
+      so[tid] = p.scale * (kPre ? aq * s_rq + u * s_kq : aq + u * s_kq);
     }
-  }
+    __syncthreads();
 
-  float4 yk = make_float4(0.f, 0.f, 0.f, 0.f), yq = yk;
+    const float4 u4 = reinterpret_cast<const float4*>(su)[cg];
+  #pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      const int r = r0 + RPP * i;
+      const float kr = sk[r] * rk;
+      s[i].x += kr * u4.x; s[i].y += kr * u4.y; s[i].z += kr * u4.z; s[i].w += kr * u4.w;
+      if (commit && tk == K - 1) __stcs(reinterpret_cast<float4*>(S + (size_t)r * DV) + cg, s[i]);
+    }
+    if (p.position_states) {  // the state after this token, for rollback
+      float* P = p.position_states + row * (size_t)(DK * DV);
 #pragma unroll
-  for (int i = 0; i < NP; ++i) {
-    const int r = r0 + RPP * i;
-    const float a = sa[r], kr = sk[r], qr = sq[r];
-    s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
-    yk.x += s[i].x * kr; yk.y += s[i].y * kr; yk.z += s[i].z * kr; yk.w += s[i].w * kr;
-    yq.x += s[i].x * qr; yq.y += s[i].y * qr; yq.z += s[i].z * qr; yq.w += s[i].w * qr;
-  }
-  reinterpret_cast<float4*>(red_k[r0])[cg] = yk;
-  reinterpret_cast<float4*>(red_q[r0])[cg] = yq;
-  __syncthreads();
+      for (int i = 0; i < NP; ++i) __stcs(reinterpret_cast<float4*>(P + (size_t)(r0 + RPP * i) * DV) + cg, s[i]);
+    }
 
-  float beta = to_f32(static_cast<const T*>(p.beta)[row]);
-  if (kPre && (p.flags & KDA_FLAG_BETA_LOGITS)) beta = 1.f / (1.f + expf(-beta));  // beta = sigmoid(b)
-  const float rk = kPre ? s_rk : 1.f;
-  if (tid < DV) {
-    float ak = 0.f, aq = 0.f;
-#pragma unroll
-    for (int r = 0; r < RPP; ++r) { ak += red_k[r][tid]; aq += red_q[r][tid]; }
-    const float vj = to_f32(static_cast<const T*>(p.v)[row * DV + tid]);
-    const float u = beta * (vj - ak * rk);
-    su[tid] = u;
-    so[tid] = p.scale * (kPre ? aq * s_rq + u * s_kq : aq + u * s_kq);
-  }
-  __syncthreads();
-
-  const float4 u4 = reinterpret_cast<const float4*>(su)[cg];
-#pragma unroll
-  for (int i = 0; i < NP; ++i) {
-    const int r = r0 + RPP * i;
-    const float kr = sk[r] * rk;
-    s[i].x += kr * u4.x; s[i].y += kr * u4.y; s[i].z += kr * u4.z; s[i].w += kr * u4.w;
-    __stcs(reinterpret_cast<float4*>(S + (size_t)r * DV) + cg, s[i]);
-  }
-
-  T* op = static_cast<T*>(p.out) + row * DV;
-  if (p.gate == nullptr) {
-    if (tid < DV) op[tid] = from_f32<T>(so[tid]);
-    return;
-  }
-  // head-wise RMSNorm over dv, then the sigmoid gate
-  float o = 0.f;
-  if (tid < DV) {
-    o = so[tid];
-    float ss = o * o;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    if ((tid & 31) == 0) s_ss[tid >> 5] = ss;
-  }
-  __syncthreads();
-  if (tid < DV) {
-    float tot = 0.f;
-#pragma unroll
-    for (int w = 0; w < DV / 32; ++w) tot += s_ss[w];
-    const float r = rsqrtf(tot / (float)DV + p.eps);
-    const float wj = p.norm_weight ? p.norm_weight[tid] : 1.0f;
-    const float gl = to_f32(static_cast<const T*>(p.gate)[row * DV + tid]);
-    const float sig = 1.0f / (1.0f + expf(-gl));
-    op[tid] = from_f32<T>(o * r * wj * sig);
+    T* op = static_cast<T*>(p.out) + row * DV;
+    if (p.gate == nullptr) {
+      if (tid < DV) op[tid] = from_f32<T>(so[tid]);
+      continue;
+    }
+    // head-wise RMSNorm over dv, then the sigmoid gate
+    float o = 0.f;
+    if (tid < DV) {
+      o = so[tid];
+      float ss = o * o;
+  #pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      if ((tid & 31) == 0) s_ss[tid >> 5] = ss;
+    }
+    __syncthreads();
+    if (tid < DV) {
+      float tot = 0.f;
+  #pragma unroll
+      for (int w = 0; w < DV / 32; ++w) tot += s_ss[w];
+      const float r = rsqrtf(tot / (float)DV + p.eps);
+      const float wj = p.norm_weight ? p.norm_weight[tid] : 1.0f;
+      const float gl = to_f32(static_cast<const T*>(p.gate)[row * DV + tid]);
+      const float sig = 1.0f / (1.0f + expf(-gl));
+      op[tid] = from_f32<T>(o * r * wj * sig);
+    }
   }
 }
 
@@ -209,6 +221,8 @@ cudaError_t launch_decode(const kda_decode_args& a, cudaStream_t stream) {
   p.state = a.state;
   p.state_indices = a.state_indices;
   p.out = a.out;
+  p.position_states = a.position_states;
+  p.tokens = a.tokens > 0 ? a.tokens : 1;
   p.H = a.H;
   p.num_slots = a.num_slots;
   p.scale = a.scale;

@@ -168,6 +168,11 @@ def test_decode_validation(L):
     assert f(N=-1) == B.KDA_ERR_INVALID_ARGUMENT
     assert f(N=0) == B.KDA_OK                                  # nothing to do, nothing launched
     assert L.kda_read_device_error(None, None) == B.KDA_ERR_INVALID_ARGUMENT
+    # multi-token decode: K >= 0 (0 means 1), position states 16-byte aligned
+    assert f(tokens=-1) == B.KDA_ERR_INVALID_ARGUMENT
+    assert f(tokens=4, position_states=FAKE + 8) == B.KDA_ERR_INVALID_ARGUMENT
+    assert f(N=0, tokens=8) == B.KDA_OK
+    assert f(N=1 << 20, H=64, tokens=64, num_slots=1 << 20) == B.KDA_ERR_UNSUPPORTED  # N K H > 2^31
 
 
 def _count(L, a):
