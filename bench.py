@@ -59,6 +59,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-snapshots", action="store_true")
     ap.add_argument("--no-preprocess", action="store_true")
+    ap.add_argument("--no-unbounded", action="store_true")
     return ap.parse_args()
 
 
@@ -348,6 +349,11 @@ def run_ours(args):
     if not args.no_preprocess:
         prep = run_preprocess(args, L, stream, dev, kern_ms, rank, w, peaks)
 
+    # ---------------- what the decay bound buys: the batch with unbounded (negative-softplus) decay
+    unb = None
+    if not args.no_unbounded:
+        unb = run_unbounded(args, L, stream, dev, kern_ms, rank, w)
+
     # ---------------- decode workload
     decode = None
     decode_multi = None
@@ -382,7 +388,8 @@ def run_ours(args):
                        "l2": f"inputs {input_bytes / 2**20:.0f} MiB per step > 126 MiB L2; no flush"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_call * args.steps, "clocks": clk, "decode": decode,
-            "snapshots": snaps, "preprocess": prep, "decode_multi": decode_multi}
+            "snapshots": snaps, "preprocess": prep, "decode_multi": decode_multi,
+            "unbounded_decay": unb}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -567,6 +574,48 @@ def run_decode(args, dev, stream, rank, world, peaks, peak_src, clocks):
                          "alg_bytes_per_launch": state_bytes, "kernel_ms": kern_ms,
                          "kernel_source_sha1": sha},
             "gpu_launches": steps}
+
+
+def run_unbounded(args, L, stream, dev, bounded_ms, rank, w):
+    """The headline batch with g = -softplus(a) (no lower bound) through KDA_FLAG_UNBOUNDED_DECAY:
+    the exact fp32 path with pairwise Gram blocks.  Its time over the bounded tensor-core launch
+    is what the g >= -5 bound buys."""
+    import torch
+    import linear_attention_serving_rule_b200 as kda
+    from linear_attention_serving_rule_b200 import binding as B
+    from linear_attention_serving_rule_b200 import synth
+    inp = synth.make_workload(WORKLOAD, device=dev, seed=rank_seed(w["seed"], rank), decay="softplus")
+    out = torch.empty_like(inp.v)
+    fin = torch.empty((w["B"], w["H"], w["dk"], w["dv"]), dtype=torch.float32, device=dev)
+    a, keep = kda.make_chunk_args(inp.q, inp.k, inp.v, inp.g, inp.beta, gate=inp.gate,
+                                  cu_seqlens=inp.cu_seqlens, out=out, final_state=fin,
+                                  flags=kda.KDA_FLAG_UNBOUNDED_DECAY)
+    nb = kda.kda_chunk_fwd_workspace_size(a)
+    ws = torch.zeros(nb, dtype=torch.uint8, device=dev)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), nb
+    sptr = stream.cuda_stream
+
+    def call():
+        rc = L.kda_chunk_fwd(ctypes.byref(a), sptr)
+        if rc != 0:
+            raise B.KdaError(rc, "kda_chunk_fwd")
+    call()
+    n = 3
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    torch.cuda.synchronize(dev)
+    for i in range(n):
+        ev[i][0].record(stream)
+        call()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    st = kda.kda_read_device_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error on the unbounded path: {kda.kda_status_string(st)}")
+    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    del keep
+    return {"decay": "g = -softplus(a), a ~ N(0,1)", "path": "fp32 CUDA cores, pairwise Gram blocks",
+            "launches": n, "kernel_ms": ms, "bounded_kernel_ms": bounded_ms,
+            "speedup_of_bound": ms / bounded_ms}
 
 
 def run_decode_multi(args, dev, stream, rank, peaks, single_ms, K=4):

@@ -90,6 +90,14 @@ typedef enum kda_dtype {
 #define KDA_FLAG_QK_L2NORM 0x20u   /* q, k L2-normalised per (token, head): x / sqrt(sum_i x_i^2 + 1e-6) */
 #define KDA_L2NORM_EPS 1e-6f
 #define KDA_FLAG_DECODE_NO_COMMIT 0x40u /* decode: leave `state` unchanged (verify pass; see tokens) */
+/* Unbounded decay: g may be any value <= 0, as with the negative-softplus decay g = -log(1 + e^a)
+ * that K3's bounded sigmoid replaced ("Kimi K3 Architecture Explained", section "Token mixing";
+ * "Kimi K3 from Moonshot AI", section "Kimi Delta Attention (KDA)").  Prefill then runs on the
+ * fp32 CUDA-core kernel with the intra-chunk Gram blocks formed pair by pair (no factor above 1),
+ * since the tensor-core tiles rely on the bound; decode handles any g.  With
+ * KDA_FLAG_CHECK_DECAY only g > 0 (or NaN) is reported.  The difference in speed between this
+ * path and the default one is what the bound buys. */
+#define KDA_FLAG_UNBOUNDED_DECAY 0x80u
 
 /* ------------------------------------------------------------------------------------------
  * Chunkwise prefill.

@@ -8,6 +8,7 @@ synthetic-input generator (synth.py).
 from .binding import (  # noqa: F401
     KDA_BF16, KDA_F32, KDA_FLAG_CHECK_DECAY, KDA_FLAG_FORCE_SIMT, KDA_FLAG_TEST_FORCE_TIMEOUT,
     KDA_FLAG_G_LOGITS, KDA_FLAG_BETA_LOGITS, KDA_FLAG_QK_L2NORM, KDA_FLAG_DECODE_NO_COMMIT,
+    KDA_FLAG_UNBOUNDED_DECAY,
     KDA_OK, KdaError, kda_chunk_fwd, kda_chunk_fwd_workspace_size, kda_decode_step,
     kda_read_device_error, kda_status_string, lib, lib_path, make_chunk_args, kda_chunk_fwd_noalloc,
     kda_chunk_fwd_snapshot_count, snapshot_count)

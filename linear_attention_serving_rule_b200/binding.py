@@ -38,6 +38,7 @@ KDA_FLAG_G_LOGITS = 0x8       # g holds decay logits a: the kernels use g = -5 s
 KDA_FLAG_BETA_LOGITS = 0x10   # beta holds logits: the kernels use sigmoid(beta)
 KDA_FLAG_QK_L2NORM = 0x20     # q, k L2-normalised per (token, head) in the kernels
 KDA_FLAG_DECODE_NO_COMMIT = 0x40  # decode: leave the state unchanged (verify pass)
+KDA_FLAG_UNBOUNDED_DECAY = 0x80   # any g <= 0 (negative-softplus decay): exact fp32 prefill path
 
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_decode_step",
             "kda_read_device_error", "kda_status_string", "kda_chunk_fwd_noalloc",

@@ -241,7 +241,8 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
 
   // bf16 with dk = dv = 128 runs on the tensor cores; everything else (and the split's
   // augmented pass 1) on the fp32 CUDA-core kernel.
-  const bool use_tc = a->dtype == KDA_BF16 && a->dk == 128 && a->dv == 128 && !(a->flags & KDA_FLAG_FORCE_SIMT);
+  const bool use_tc = a->dtype == KDA_BF16 && a->dk == 128 && a->dv == 128 &&
+                      !(a->flags & (KDA_FLAG_FORCE_SIMT | KDA_FLAG_UNBOUNDED_DECAY));
 
   // Pass 1 of split sequences: the head segment from the true initial state, and the
   // other non-final segments from [0 | I] (local state and transition matrix).

@@ -20,6 +20,11 @@
 //
 // AUG = true runs the split pass 1 on the augmented state [S | M] (dv + dk columns) with
 // values augmented by zeros, so M accumulates the segment's transition matrix.
+//
+// With KDA_FLAG_UNBOUNDED_DECAY the decay may be any g <= 0 (the negative-softplus decay of
+// Kimi Linear, which K3 replaced by the bounded sigmoid: "Kimi K3 Architecture Explained",
+// section "Token mixing"), so e^{-gamma} may overflow.  A and P are then formed pair by pair
+// with e^{gamma_t - gamma_s} <= 1 (s <= t); every other product already uses factors <= 1.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -66,6 +71,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool g_logits = (p.flags & KDA_FLAG_G_LOGITS) != 0;
   const bool b_logits = (p.flags & KDA_FLAG_BETA_LOGITS) != 0;
   const bool l2norm = (p.flags & KDA_FLAG_QK_L2NORM) != 0;
+  const bool unbounded = (p.flags & KDA_FLAG_UNBOUNDED_DECAY) != 0;
   const bool write_out = (seg.role == kRoleWhole || seg.role == kRoleFromWs);
 
   // ---- start state
@@ -102,7 +108,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const size_t r = ((size_t)(seg.tok0 + c0 + t) * H + h) * DK + c;
         qx = to_f32(q[r]); kx = to_f32(k[r]); gx = to_f32(g[r]);
         if (g_logits) gx = KDA_G_MIN / (1.f + expf(-gx));  // g = g_min sigmoid(a)
-        if (checked && !(gx >= KDA_G_MIN && gx <= 0.f)) report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
+        if (checked && !((unbounded || gx >= KDA_G_MIN) && gx <= 0.f))
+          report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
       }
       sm.Qt[idx] = qx; sm.Kt[idx] = kx; sm.G[idx] = gx;
     }
@@ -136,30 +143,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int t = 0; t < kC; ++t) {
         gam += sm.G[t * DK + c];
         sm.G[t * DK + c] = gam;
-        const float e = expf(gam), ei = expf(-gam);
+        const float e = expf(gam);
         const float kx = sm.Kt[t * DK + c];
-        sm.Kb[t * LDB + c] = kx * ei;
+        // unbounded decay: Kb keeps the raw q for the pairwise Gram blocks
+        sm.Kb[t * LDB + c] = unbounded ? sm.Qt[t * DK + c] : kx * expf(-gam);
         sm.Kt[t * DK + c] = kx * e;
         sm.Qt[t * DK + c] *= e;
         sm.Kh[t * DK + c] = kx;  // raw k, scaled below once gamma_C is known
       }
       sm.eC[c] = expf(gam);
-      for (int t = 0; t < kC; ++t) sm.Kh[t * DK + c] *= expf(gam - sm.G[t * DK + c]);
+      if (!unbounded)
+        for (int t = 0; t < kC; ++t) sm.Kh[t * DK + c] *= expf(gam - sm.G[t * DK + c]);
     }
     __syncthreads();
     // ---- decayed Gram blocks A (strict) and P (inclusive): one (t, s) pair per thread
     {
       const int t = tid / kC, s = tid % kC;
       float a = 0.f, pp = 0.f;
-      for (int c = 0; c < DK; ++c) {
-        const float kb = sm.Kb[s * LDB + c];
-        a += sm.Kt[t * DK + c] * kb;
-        pp += sm.Qt[t * DK + c] * kb;
+      if (!unbounded) {
+        for (int c = 0; c < DK; ++c) {
+          const float kb = sm.Kb[s * LDB + c];
+          a += sm.Kt[t * DK + c] * kb;
+          pp += sm.Qt[t * DK + c] * kb;
+        }
+      } else if (s <= t) {  // raw k (Kh), raw q (Kb) and e^{gamma_t - gamma_s} <= 1
+        for (int c = 0; c < DK; ++c) {
+          const float f = expf(sm.G[t * DK + c] - sm.G[s * DK + c]);
+          const float ks = sm.Kh[s * DK + c];
+          a += sm.Kh[t * DK + c] * ks * f;
+          pp += sm.Kb[t * LDB + c] * ks * f;
+        }
       }
       sm.A[t * kC + s] = (s < t) ? a : 0.f;
       sm.P[t * kC + s] = (s <= t) ? pp : 0.f;
     }
     __syncthreads();
+    if (unbounded) {  // now K e^{gamma_C - gamma}
+      if (tid < DK) {
+        const float gC = sm.G[(kC - 1) * DK + tid];
+        for (int t = 0; t < kC; ++t) sm.Kh[t * DK + tid] *= expf(gC - sm.G[t * DK + tid]);
+      }
+      __syncthreads();
+    }
     // ---- T' = (I + Diag(beta) A)^-1 Diag(beta): lane j solves column j
     if (tid < kC) {
       const int j = tid;

@@ -94,7 +94,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
       sq[i] = to_f32(qp[i]);
       float gi = to_f32(gp[i]);
       if (g_logits) gi = KDA_G_MIN / (1.f + expf(-gi));  // g = g_min sigmoid(a)
-      if (checked && !(gi >= KDA_G_MIN && gi <= 0.0f)) report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
+      if (checked && !(((p.flags & KDA_FLAG_UNBOUNDED_DECAY) || gi >= KDA_G_MIN) && gi <= 0.0f))
+        report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
       sa[i] = expf(gi);
     }
     __syncthreads();

@@ -95,13 +95,14 @@ def _randn(shape, gen, device):
 def make_prefill(*, H: int, dk: int, dv: int, dtype="bf16", seed: int = 0,
                  device="cpu", lengths=None, B: int | None = None, T: int | None = None,
                  gate: bool = True, init_state: bool = False, decay_shift: float = 0.0,
-                 state_std: float = 0.02, raw: bool = False) -> PrefillInputs:
+                 state_std: float = 0.02, raw: bool = False, decay: str = "sigmoid") -> PrefillInputs:
     """Packed prefill inputs.  Give either `lengths` (varlen) or B and T (B equal
     sequences of T tokens, stored packed as [B*T, H, d]).
 
     raw=True returns the same draws before their last step: q and k not L2-normalised, beta
     and g as the logits b and a of beta = sigmoid(b), g = -5 sigmoid(a) (the inputs of the
-    library's pre-processing flags)."""
+    library's pre-processing flags).  decay="softplus" draws g = -softplus(a) instead of
+    -5 sigmoid(a): the unbounded negative-softplus decay (no lower bound)."""
     if lengths is None:
         lengths = np.full(B, T, dtype=np.int64)
     cu = cu_from_lengths(lengths)
@@ -117,7 +118,12 @@ def make_prefill(*, H: int, dk: int, dv: int, dtype="bf16", seed: int = 0,
     b_logit = _randn((T_tot, H), gen, device)
     beta = (b_logit if raw else torch.sigmoid(b_logit)).to(dt)
     a_logit = _randn((T_tot, H, dk), gen, device) + decay_shift
-    g = (a_logit if raw else G_MIN * torch.sigmoid(a_logit)).to(dt)
+    if raw:
+        g = a_logit.to(dt)
+    elif decay == "softplus":
+        g = (-torch.nn.functional.softplus(a_logit)).to(dt)
+    else:
+        g = (G_MIN * torch.sigmoid(a_logit)).to(dt)
     gt = _randn((T_tot, H, dv), gen, device).to(dt) if gate else None
     s0 = (state_std * _randn((N, H, dk, dv), gen, device)) if init_state else None
     return PrefillInputs(q, k, v, g, beta, gt, s0, cu)
@@ -133,7 +139,8 @@ def make_workload(name: str, device="cpu", **overrides) -> PrefillInputs:
     return make_prefill(H=w["H"], dk=w["dk"], dv=w["dv"], dtype=w["dtype"], seed=w["seed"],
                         device=device, lengths=lengths, B=w.get("B"), T=w.get("T"),
                         gate=w["gate"], init_state=w["init_state"],
-                        decay_shift=w.get("decay_shift", 0.0), raw=w.get("raw", False))
+                        decay_shift=w.get("decay_shift", 0.0), raw=w.get("raw", False),
+                        decay=w.get("decay", "sigmoid"))
 
 
 @dataclass
