@@ -25,18 +25,19 @@
 // handed back right after the decay scan), k and q (landing interleaved as one 128-row tile;
 // handed back after the UMMAs that read their in-place products) and v (after W/U').  Warps 0-7
 // are two compute warpgroups; warp w owns TMEM lane quarter w % 4.  Decay prep, Gram read-out,
-// UT inverse and the -W / U conversions run on all 256 threads; in the shadow of the Gram UMMAs
-// both warpgroups run the previous chunk's epilogue; while warps 0-1 invert the diagonal blocks
-// of the UT transform, warps 2-7 make the bf16 copy of the state; in the shadow of the U and O
-// UMMAs all warps decay the state and scan the next chunk's decay.  Off-diagonal blocks of the
-// inverse are warp-level tf32 MMAs.  Thread 0 issues the UMMAs.  The gate logits are staged
-// from global memory with cp.async.
+// UT inverse and the -W / U conversions run on all 256 threads; in the shadow of the Gram and of
+// the W|U' UMMAs both warpgroups run the previous chunk's epilogue; while warps 0-1 invert the
+// diagonal blocks of the UT transform, warps 2-7 make the bf16 copy of the state; in the shadow
+// of the U and O UMMAs all warps decay the state and scan the next chunk's decay.  Off-diagonal
+// blocks of the inverse are warp-level tf32 MMAs.  Thread 0 issues the UMMAs.  The gate logits
+// are staged from global memory with cp.async into their own buffer.
 //
 // TMEM (512 columns allocated): [0,128) the fp32 state S (M=128; decayed in place while the
 // U and O UMMAs run, then K^T U accumulated onto it); [128,288) A|P (M=128, N=160);
-// [288,352) W -> O and [352,416) U' -> U: each M=64 product is issued as two N=64 halves, columns
-// 0-63 at lane offset 0 and columns 64-127 at lane offset 16 of the same TMEM columns, so a warp's
-// 32 lanes read 16 rows x 2 column halves and every lane takes part in the read-outs.
+// [288,352) W, [352,416) U' -> U and [416,480) O: each M=64 product is issued as two N=64 halves,
+// columns 0-63 at lane offset 0 and columns 64-127 at lane offset 16 of the same TMEM columns, so
+// a warp's 32 lanes read 16 rows x 2 column halves and every lane takes part in the read-outs.
+// O keeps its own columns so that a chunk's epilogue can run beside the next chunk's UMMAs.
 //
 // Every wait is bounded (%globaltimer): on expiry the kernel records KDA_ERR_TIMEOUT, stops
 // issuing work, drains its own in-flight TMA and UMMA operations (bounded again), frees TMEM
@@ -69,14 +70,16 @@ constexpr uint32_t OFF_S = 155648;   // bf16 state, MN-major [dk rows][dv], two 
 constexpr uint32_t OFF_TP = 188416;  // T' = T Diag(beta), bf16 [64][64]
 constexpr uint32_t OFF_P = 196608;   // P (causally masked), bf16 [64][64]
 constexpr uint32_t OFF_MISC = 204800;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 8192 + 1024;
+constexpr uint32_t OFF_GATE = OFF_MISC + 8192;  // gate logits of the chunk whose epilogue is pending
+constexpr uint32_t SMEM_BYTES = OFF_GATE + 16384 + 1024;
+static_assert(SMEM_BYTES <= 232448, "over the 227 KB of shared memory a block may use");
 // fp32 L = Diag(beta) A [64][68], then fp32 T [64][68]: a row stride of 4 mod 32 words keeps the
 // mma.sync A-fragment loads (8 rows x 4 columns per warp) free of bank conflicts
 constexpr int LDF = 68;
 constexpr int LDT = 68;
 constexpr uint32_t OFF_TF = OFF_KC + 64 * LDF * 4;
 
-constexpr uint32_t TM_S = 0, TM_AP = 128, TM_WU = 288;
+constexpr uint32_t TM_S = 0, TM_AP = 128, TM_WU = 288, TM_O = 416;
 
 // The column operands Kc_0..Kc_3 (16(a+1) rows each) are stacked into one 160-row K-major tile
 // (two 64-column blocks of 160 x 128 bytes); Kc_a starts at row ap_off(a), which is also the
@@ -370,13 +373,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
     }
 
-    // Epilogue of one chunk: O sits at TMEM lane offset 0 of [288,416) until the next chunk's
-    // W/U' UMMAs, so it runs in the shadow of the next chunk's Gram UMMAs.  Lanes < 16 of each
-    // warp hold the 64 O rows; the two warpgroups hold the two column halves and exchange their
-    // partial sums of squares; the gate logits come from the staging copy made by load_gate.
-    // The gate logits of a chunk are staged with cp.async into the T'/P region, which is free from
-    // the start of the next chunk until its Gram read-out; row t at OFF_TP + 256 t, 16-byte chunk c
-    // at position c ^ (t & 15).
+    // The gate logits of a chunk are staged with cp.async at the start of the next chunk, into
+    // their own buffer: row t at OFF_GATE + 256 t, 16-byte chunk c at position c ^ (t & 15).
     auto load_gate = [&](int L_e, int32_t tok_e) {
       if (!has_gate) return;
 #pragma unroll
@@ -384,20 +382,45 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int idx = tid + kCompute * r;
         const int t = idx >> 4, c16 = idx & 15;
         if (t < L_e)
-          cp_async_16(sm_u + OFF_TP + t * 256 + ((c16 ^ (t & 15)) << 4),
+          cp_async_16(sm_u + OFF_GATE + t * 256 + ((c16 ^ (t & 15)) << 4),
                       static_cast<const __nv_bfloat16*>(p.gate) + ((size_t)(tok_e + t) * H + h) * DV + 8 * c16);
       }
       cp_async_commit();
     };
-    // Epilogue of one chunk, run by both warpgroups: lanes l < 16 of warp (q, wg) hold columns
-    // 32 wg .. 32 wg + 31 and lanes l + 16 columns 64 + 32 wg .. of O row 16 q + l; a row's sum of
-    // squares is combined across the two lanes with a shuffle and across the warpgroups through
-    // shared memory.  The gate logits come from the cp.async staging.
-    auto epilogue = [&](int L_e, int32_t tok_e) {
+    // Epilogue of one chunk, run by both warpgroups in two parts while the next chunk's UMMAs run:
+    // O stays in TMEM columns [416,480) until the next chunk's O UMMAs.  Lanes l < 16 of warp
+    // (q, wg) hold columns 32 wg .. 32 wg + 31 and lanes l + 16 columns 64 + 32 wg .. of O row
+    // 16 q + l; a row's sum of squares is combined across the two lanes with a shuffle and across
+    // the warpgroups through shared memory.  Part A (beside the Gram UMMAs) finds the row scale
+    // and writes the thread's first 16 columns, part B (beside the W|U' UMMAs) the other 16.
+    float epi_sc = 0.f;  // scale / rms of the thread's O row, from part A to part B
+    auto epi_store = [&](int L_e, int32_t tok_e, const uint32_t* v, int oc0) {
       const int t = 16 * q4 + (lane & 15);
+      if (t >= L_e) return;
       const int c0 = 64 * (lane >> 4) + 32 * wg;
+      uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ((size_t)(tok_e + t) * H + h) * DV + c0);
+#pragma unroll
+      for (int oc = 0; oc < 2; ++oc) {
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]) * epi_sc;
+        if (has_gate) {
+          float gl8[8];
+          const int c16 = (c0 >> 3) + oc0 + oc;
+          unpack8(at16(sm, OFF_GATE + t * 256 + ((c16 ^ (t & 15)) << 4)), gl8);
+          const float4 w0 = *reinterpret_cast<const float4*>(&m->nw[c0 + 8 * (oc0 + oc)]);
+          const float4 w1 = *reinterpret_cast<const float4*>(&m->nw[c0 + 8 * (oc0 + oc) + 4]);
+          const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] *= __fdividef(w[e], 1.f + ex2(-gl8[e] * kLog2e));
+        }
+        op[oc0 + oc] = pack8(f);
+      }
+    };
+    auto epilogue_a = [&](int L_e, int32_t tok_e) {
+      const int t = 16 * q4 + (lane & 15);
       uint32_t v[32];
-      tmem_ld32(tl + TM_WU + 32 * wg, v);
+      tmem_ld32(tl + TM_O + 32 * wg, v);
       tmem_wait_ld();
       float ss = 0.f;
 #pragma unroll
@@ -409,27 +432,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane < 16) m->ssq[wg][t] = ss;
       sync_wg();
       ss += m->ssq[wg ^ 1][t];
-      if (t >= L_e) return;
       const float rr = has_gate ? rsqrtf(ss * p.scale * p.scale / (float)DV + p.eps) : 1.f;
-      const float sc = p.scale * rr;
-      uint4* op = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + ((size_t)(tok_e + t) * H + h) * DV + c0);
-#pragma unroll
-      for (int oc = 0; oc < 4; ++oc) {
-        float f[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]) * sc;
-        if (has_gate) {
-          float gl8[8];
-          const int c16 = (c0 >> 3) + oc;
-          unpack8(at16(sm, OFF_TP + t * 256 + ((c16 ^ (t & 15)) << 4)), gl8);
-          const float4 w0 = *reinterpret_cast<const float4*>(&m->nw[c0 + 8 * oc]);
-          const float4 w1 = *reinterpret_cast<const float4*>(&m->nw[c0 + 8 * oc + 4]);
-          const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] *= __fdividef(w[e], 1.f + ex2(-gl8[e] * kLog2e));
-        }
-        op[oc] = pack8(f);
-      }
+      epi_sc = p.scale * rr;
+      epi_store(L_e, tok_e, v, 0);
+    };
+    auto epilogue_b = [&](int L_e, int32_t tok_e) {
+      uint32_t v[16];
+      tmem_ld16(tl + TM_O + 32 * wg + 16, v);
+      tmem_wait_ld();
+      epi_store(L_e, tok_e, v, 2);
     };
     // bf16 copy of the state S for the UMMAs: 64-column halves [hb0, hb1) of this warp's 32 rows;
     // with snap != null also the fp32 snapshot of S
@@ -633,7 +644,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the previous chunk's epilogue (its O is still in TMEM)
       cp_async_wait_all();
       sync_wg();  // the staged gate logits are visible to every thread
-      if (write_out && j > 0) epilogue(L_prev, tok_prev);
+      if (write_out && j > 0) epilogue_a(L_prev, tok_prev);
       {
         const bool r = wg_wait(&m->mma, mph & 1u);
         ++mph;
@@ -822,7 +833,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                       false);
         }
       }
-      if (!mma_commit_wait()) { ok = false; break; }
+      if (tid == 0) umma_commit(&m->mma);
+      if (write_out && j > 0) epilogue_b(L_prev, tok_prev);  // in the shadow of the W|U' UMMAs
+      {
+        const bool r = wg_wait(&m->mma, mph & 1u);
+        ++mph;
+        tc_fence_after();
+        if (!r) { ok = false; break; }
+      }
       if (tid == 0 && need_v) mbar_arrive(&m->empty_v);
 
       // ---------------------------------------------------------------- -W -> bf16
@@ -850,8 +868,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_k_loop(tmem + TM_WU + 64, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S, 16384, false, 0, 8, id, need_v);
         umma_k_loop(tmem + TM_WU + 64 + hi, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S + 16384, 16384, false, 0, 8,
                     id, need_v);
-        umma_k_loop(tmem + TM_WU, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S, 16384, false, 0, 8, id, false);
-        umma_k_loop(tmem + TM_WU + hi, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S + 16384, 16384, false, 0, 8,
+        umma_k_loop(tmem + TM_O, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S, 16384, false, 0, 8, id, false);
+        umma_k_loop(tmem + TM_O + hi, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S + 16384, 16384, false, 0, 8,
                     id, false);
         umma_commit(&m->mma);
       }
@@ -907,9 +925,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------------- UMMA: O += P U ; S += Kh^T U
       if (tid == 0) {
         tc_fence_after();
-        umma_k_loop(tmem + TM_WU, sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL, 8192, false, 0, 4,
+        umma_k_loop(tmem + TM_O, sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL, 8192, false, 0, 4,
                     idesc_bf16_f32(64, 64, 0, 1), true);
-        umma_k_loop(tmem + TM_WU + (16u << 16), sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL + 8192, 8192, false, 0, 4,
+        umma_k_loop(tmem + TM_O + (16u << 16), sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL + 8192, 8192, false, 0, 4,
                     idesc_bf16_f32(64, 64, 0, 1), true);
         umma_k_loop(tmem + TM_S, sm_u + OFF_KH, 8192, false, 0, sm_u + OFF_KL, 8192, false, 0, 4,
                     idesc_bf16_f32(128, 128, 1, 1), true);
@@ -923,7 +941,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       load_gate(L_prev, tok_prev);
       cp_async_wait_all();
       sync_wg();
-      epilogue(L_prev, tok_prev);
+      epilogue_a(L_prev, tok_prev);
+      epilogue_b(L_prev, tok_prev);
     }
 
     // ---------------------------------------------------------------- end state
