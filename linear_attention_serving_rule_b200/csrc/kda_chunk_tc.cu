@@ -21,7 +21,7 @@
 // operand Kc_a = k e^{r_a - gamma} over the first 16(a+1) tokens; one M=128 UMMA per a
 // produces A (rows 0-63) and P (rows 64-127) from the stacked operand [k; q] e^{gamma - r_own}.
 //
-// Work split (288 threads): warp 8 is the TMA producer with three groups of tiles: g (with beta,
+// Work split (320 threads): warp 8 is the TMA producer with three groups of tiles: g (with beta,
 // handed back right after the decay scan), k and q (landing interleaved as one 128-row tile;
 // handed back after the UMMAs that read their in-place products) and v (after W/U').  Warps 0-7
 // are two compute warpgroups; warp w owns TMEM lane quarter w % 4.  Decay prep, Gram read-out,
@@ -29,8 +29,9 @@
 // the W|U' UMMAs both warpgroups run the previous chunk's epilogue; while warps 0-1 invert the
 // diagonal blocks of the UT transform, warps 2-7 make the bf16 copy of the state; in the shadow
 // of the U and O UMMAs all warps decay the state and scan the next chunk's decay.  Off-diagonal
-// blocks of the inverse are warp-level tf32 MMAs.  Thread 0 issues the UMMAs.  The gate logits
-// are staged from global memory with cp.async into their own buffer.
+// blocks of the inverse are warp-level tf32 MMAs.  Warp 9 issues the UMMAs: the compute warps
+// publish each group's operands on an mbarrier and go on with the work beside it.  The gate
+// logits are staged from global memory with cp.async into their own buffer.
 //
 // TMEM (512 columns allocated): [0,128) the fp32 state S (M=128; decayed in place while the
 // U and O UMMAs run, then K^T U accumulated onto it); [128,288) A|P (M=128, N=160);
@@ -43,6 +44,7 @@
 // issuing work, drains its own in-flight TMA and UMMA operations (bounded again), frees TMEM
 // and returns.
 #include <cuda.h>
+#include <cstddef>
 
 #include "kda_internal.cuh"
 #include "ptx_sm100.cuh"
@@ -56,7 +58,7 @@ constexpr int C = 64;
 constexpr int DK = 128;
 constexpr int DV = 128;
 constexpr int kCompute = 256;
-constexpr int kThreads = 288;
+constexpr int kThreads = 320;  // 8 compute warps, the TMA producer (warp 8), the UMMA issuer (warp 9)
 constexpr float kLog2e = 1.4426950408889634f;
 
 // shared memory map (bytes from a 1024-aligned base)
@@ -88,17 +90,19 @@ __host__ __device__ constexpr uint32_t ap_off(int a) { return a == 0 ? 0u : a ==
 constexpr uint32_t KC_ROWS = 160, KC_BLK = KC_ROWS * 128;
 
 struct Misc {
-  uint64_t full_g, full_kq, full_v, empty_g, empty_kq, empty_v, mma;
+  uint64_t full_g, full_kq, full_v, empty_g, empty_kq, empty_v, mma, ops;
   uint32_t tmem_base;
   int32_t abort;
   float beta[2][C];  // double-buffered by chunk parity (written by the producer warp)
   float se[4][DK];  // e^{decay over sub-tile m}; channel 8o + e at [m][16 e + o]
   float ec[DK];     // e^{gamma_C}
-  float nw[DV];     // RMSNorm weight (1 without one)
+  alignas(16) float nw[DV];  // RMSNorm weight (1 without one); read as float4
   float ssq[2][C];  // epilogue: per-row sums of squares of the two column halves
   float qkss[2][2 * C];  // with KDA_FLAG_QK_L2NORM: sums of squares of the k|q rows, by column half
 };
 static_assert(sizeof(Misc) <= 8192, "misc block too large");
+static_assert(offsetof(Misc, nw) % 16 == 0, "float4 reads of the norm weight need 16-byte alignment");
+static_assert(offsetof(Misc, full_g) % 8 == 0, "mbarriers need 8-byte alignment");
 
 struct TcMaps {
   CUtensorMap q, k, g, v;
@@ -184,25 +188,40 @@ __device__ __forceinline__ void mma_3xtf32(float (&d)[3][4], const float (&a)[4]
   mma_tf32(d[2], al, bh);
 }
 
-// Issue the K loop of one UMMA.  K-major operands step 32 bytes per 16-wide K step and jump to
-// their second 64-column block (blk bytes away) after 4 steps; MN-major ones step 2048 bytes.
-// The descriptors are built once; each K step only adds its byte offset / 16 to the start-address
-// field (bits 0-13), which cannot carry out for shared-memory addresses.
-__device__ __forceinline__ void umma_k_loop(uint32_t d, uint32_t a_addr, uint32_t a_lbo, bool a_kmajor,
-                                            uint32_t a_blk, uint32_t b_addr, uint32_t b_lbo, bool b_kmajor,
-                                            uint32_t b_blk, int ksteps, uint32_t idesc, bool accumulate) {
-  const uint64_t a0 = smem_desc_sw128(a_addr, a_lbo, 1024);
-  const uint64_t b0 = smem_desc_sw128(b_addr, b_lbo, 1024);
+// One accumulation chain of a UMMA group: destination, descriptors (built once), operand majors
+// and 64-column block strides.  K-major operands step 32 bytes per 16-wide K step and jump to their
+// second 64-column block (blk bytes away) after 4 steps; MN-major ones step 2048 bytes.  Each K
+// step only adds its byte offset / 16 to the start-address field (bits 0-13), which cannot carry
+// out for shared-memory addresses.
+struct UChain {
+  uint32_t d;
+  uint64_t a0, b0;
+  uint32_t a_blk, b_blk, idesc;
+  bool a_kmajor, b_kmajor, accumulate;
+};
+__device__ __forceinline__ UChain uchain(uint32_t d, uint32_t a_addr, uint32_t a_lbo, bool a_kmajor, uint32_t a_blk,
+                                         uint32_t b_addr, uint32_t b_lbo, bool b_kmajor, uint32_t b_blk, uint32_t idesc,
+                                         bool accumulate) {
+  return UChain{d, smem_desc_sw128(a_addr, a_lbo, 1024), smem_desc_sw128(b_addr, b_lbo, 1024), a_blk, b_blk, idesc,
+                a_kmajor, b_kmajor, accumulate};
+}
+// Issue NC independent chains of `ksteps` K steps each, interleaved step by step: the K steps of one
+// chain accumulate into the same TMEM tile and wait for each other, so the other chains' steps
+// fill the tensor pipe meanwhile (issued chain after chain, a group runs at about one step per
+// pipe latency).
+template <int NC>
+__device__ __forceinline__ void umma_interleaved(const UChain (&c)[NC], int ksteps) {
 #pragma unroll
   for (int k = 0; k < ksteps; ++k) {
-    const uint32_t ao = a_kmajor ? (uint32_t)(k >> 2) * a_blk + (uint32_t)(k & 3) * 32u : (uint32_t)k * 2048u;
-    const uint32_t bo = b_kmajor ? (uint32_t)(k >> 2) * b_blk + (uint32_t)(k & 3) * 32u : (uint32_t)k * 2048u;
-    umma_bf16(d, a0 + (ao >> 4), b0 + (bo >> 4), idesc, (accumulate || k > 0) ? 1u : 0u);
+#pragma unroll
+    for (int i = 0; i < NC; ++i) {
+      const uint32_t ao = c[i].a_kmajor ? (uint32_t)(k >> 2) * c[i].a_blk + (uint32_t)(k & 3) * 32u : (uint32_t)k * 2048u;
+      const uint32_t bo = c[i].b_kmajor ? (uint32_t)(k >> 2) * c[i].b_blk + (uint32_t)(k & 3) * 32u : (uint32_t)k * 2048u;
+      umma_bf16(c[i].d, c[i].a0 + (ao >> 4), c[i].b0 + (bo >> 4), c[i].idesc, (c[i].accumulate || k > 0) ? 1u : 0u);
+    }
   }
 }
 
-// kPre: the decay-logit and q/k L2-norm pre-processing (KDA_FLAG_G_LOGITS, KDA_FLAG_QK_L2NORM) is
-// compiled in; the instance without it keeps the plain path free of their branches.
 template <bool kPre>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ Plan plan, const __grid_constant__ TcMaps maps, const ChunkParams p) {
@@ -231,6 +250,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&m->full_g, 1); mbar_init(&m->full_kq, 1); mbar_init(&m->full_v, 1);
     mbar_init(&m->empty_g, 1); mbar_init(&m->empty_kq, 1); mbar_init(&m->empty_v, 1);
     mbar_init(&m->mma, 1);
+    mbar_init(&m->ops, 8);  // one arrival per compute warp: a UMMA group's operands are in place
     m->abort = 0;
     fence_mbar_init();
   }
@@ -300,6 +320,90 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ikq >= 0) wait_bounded(&m->full_kq, (uint32_t)(ikq & 1), m, drain_limit, p.error_word, false);
       if (iv >= 0) wait_bounded(&m->full_v, (uint32_t)(iv & 1), m, drain_limit, p.error_word, false);
     }
+  } else if (warp == 9) {
+    // ===================================================================== UMMA issuer
+    // Lane 0 issues each UMMA group once the eight compute warps have published its operands
+    // (one arrival each on m->ops) and commits it to m->mma.  Issuing blocks for as long as the
+    // tensor core takes to accept the group, so the compute warps never issue.
+    if (lane == 0) {
+      uint32_t oph = 0;
+      int committed = 0;
+      const uint32_t hi = 16u << 16;
+      for (int j = 0; j < nchunks; ++j) {
+        const uint32_t par = (uint32_t)(j & 1);
+        // A | P over the stacked Kc operand, as two N=80 halves (Kc rows 0-79 and 80-159; row 80
+        // starts a swizzle atom) whose K steps interleave
+        if (!wait_bounded(&m->ops, (oph++) & 1u, m, limit, p.error_word)) break;
+        tc_fence_after();
+        {
+          const uint32_t id = idesc_bf16_f32(128, KC_ROWS / 2, 0, 0);
+          const UChain c[2] = {
+              uchain(tmem + TM_AP, sm_u + OFF_KL, 16, true, 16384, sm_u + OFF_KC, 16, true, KC_BLK, id, false),
+              uchain(tmem + TM_AP + KC_ROWS / 2, sm_u + OFF_KL, 16, true, 16384, sm_u + OFF_KC + (KC_ROWS / 2) * 128, 16,
+                     true, KC_BLK, id, false)};
+          umma_interleaved(c, 8);
+        }
+        umma_commit(&m->mma);
+        ++committed;
+        // W | U': columns 0-63 at lane offset 0, 64-127 at lane offset 16: W in [288,352), U' in
+        // [352,416); one N=128 UMMA per half, whose B operand is [e^g k block | v block] -- two MN
+        // atoms (OFF_V - OFF_KQ) and (OFF_V + 8192 - OFF_KQ - 16384) bytes apart
+        if (!wait_bounded(&m->ops, (oph++) & 1u, m, limit, p.error_word)) break;
+        if (need_v && !wait_bounded(&m->full_v, par, m, limit, p.error_word)) break;
+        tc_fence_after();
+        if (need_v) {
+          const uint32_t id = idesc_bf16_f32(64, 128, 0, 1);
+          const UChain c[2] = {
+              uchain(tmem + TM_WU, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ, OFF_V - OFF_KQ, false, 0, id, false),
+              uchain(tmem + TM_WU + hi, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ + 16384,
+                     OFF_V + 8192 - OFF_KQ - 16384, false, 0, id, false)};
+          umma_interleaved(c, 4);
+        } else {
+          const uint32_t id = idesc_bf16_f32(64, 64, 0, 1);
+          const UChain c[2] = {
+              uchain(tmem + TM_WU, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ, 16384, false, 0, id, false),
+              uchain(tmem + TM_WU + hi, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ + 16384, 16384, false, 0, id, false)};
+          umma_interleaved(c, 4);
+        }
+        umma_commit(&m->mma);
+        ++committed;
+        // U = U' - W S0 ; O = Qt S0
+        if (!wait_bounded(&m->ops, (oph++) & 1u, m, limit, p.error_word)) break;
+        tc_fence_after();
+        {
+          const uint32_t id = idesc_bf16_f32(64, 64, 0, 1);
+          const UChain c[4] = {
+              uchain(tmem + TM_WU + 64, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S, 16384, false, 0, id, need_v),
+              uchain(tmem + TM_WU + 64 + hi, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S + 16384, 16384, false, 0, id,
+                     need_v),
+              uchain(tmem + TM_O, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S, 16384, false, 0, id, false),
+              uchain(tmem + TM_O + hi, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S + 16384, 16384, false, 0, id,
+                     false)};
+          umma_interleaved(c, 8);
+        }
+        umma_commit(&m->mma);
+        ++committed;
+        // O += P U ; S += Kh^T U
+        if (!wait_bounded(&m->ops, (oph++) & 1u, m, limit, p.error_word)) break;
+        tc_fence_after();
+        {
+          const UChain c[3] = {
+              uchain(tmem + TM_O, sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL, 8192, false, 0, idesc_bf16_f32(64, 64, 0, 1),
+                     true),
+              uchain(tmem + TM_O + hi, sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL + 8192, 8192, false, 0,
+                     idesc_bf16_f32(64, 64, 0, 1), true),
+              uchain(tmem + TM_S, sm_u + OFF_KH, 8192, false, 0, sm_u + OFF_KL, 8192, false, 0,
+                     idesc_bf16_f32(128, 128, 1, 1), true)};
+          umma_interleaved(c, 4);
+        }
+        umma_commit(&m->mma);
+        ++committed;
+      }
+      // the last group committed must finish before TMEM is freed (after an abort too)
+      if (committed > 0)
+        wait_bounded(&m->mma, (uint32_t)(committed - 1) & 1u, m, drain_limit, p.error_word, false);
+    }
+    __syncwarp();
   } else {
     // ===================================================================== compute warpgroups
     const int q4 = warp & 3;   // TMEM lane quarter
@@ -324,17 +428,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       sync_wg();
       return *(volatile int32_t*)&m->abort == 0;
     };
-    auto mma_commit_wait = [&]() -> bool {
-      if (tid == 0) umma_commit(&m->mma);
-      const bool r = wg_wait(&m->mma, mph & 1u);
-      ++mph;
-      tc_fence_after();
-      return r;
-    };
-    auto sync_for_mma = [&]() {
+    // publish this warp's operand writes (shared memory and TMEM) to the UMMA issuer
+    auto ops_arrive = [&]() {
       fence_proxy_async_smem();
       tc_fence_before();
-      sync_wg();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&m->ops);
     };
 
     // ---------------------------------------------------------------- start state -> TMEM + bf16 copy
@@ -532,7 +631,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int32_t tok = seg.tok0 + j * C;
       const uint32_t par = (uint32_t)(j & 1);
       const float* beta = m->beta[j & 1];
-      if (write_out && j > 0) load_gate(L_prev, tok_prev);  // consumed by its epilogue below
       // ---------------------------------------------------------------- decay prep: all bf16 operands
 
       if (!wg_wait(&m->full_kq, par)) { ok = false; break; }
@@ -632,14 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int si = 16 * (tid & 7) + (tid >> 3);
         m->ec[tid] = m->se[0][si] * m->se[1][si] * m->se[2][si] * m->se[3][si];
       }
-      sync_for_mma();
-      // ---------------------------------------------------------------- UMMA: A | P
-      if (tid == 0) {
-        tc_fence_after();
-        umma_k_loop(tmem + TM_AP, sm_u + OFF_KL, 16, true, 16384, sm_u + OFF_KC, 16, true, KC_BLK, 8,
-                    idesc_bf16_f32(128, KC_ROWS, 0, 0), false);
-        umma_commit(&m->mma);
-      }
+      ops_arrive();  // ---------------------------------------------- UMMA: A | P (issued by warp 9)
       // ---------------------------------------------------------------- in the shadow of the Gram UMMAs:
       // the previous chunk's epilogue (its O is still in TMEM)
       cp_async_wait_all();
@@ -809,31 +900,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           at16(sm, OFF_TP + sw128_oct(i, oc, 8192)) = pack8(f);
         }
       }
-      sync_for_mma();
-      // ---------------------------------------------------------------- UMMA: W = T' Kt, U' = T' V
-      if (tid == 0 && need_v) wait_bounded(&m->full_v, par, m, limit, p.error_word);
-      sync_wg();
-      if (*(volatile int32_t*)&m->abort) { ok = false; break; }
-      if (tid == 0) {
-        tc_fence_after();
-        // columns 0-63 at lane offset 0, 64-127 at lane offset 16: W in [288,352), U' in [352,416)
-        // with values: one N=128 UMMA per half, whose B operand is [e^g k block | v block] -- two
-        // MN atoms (OFF_V - OFF_KQ) and (OFF_V + 8192 - OFF_KQ - 16384) bytes apart -- so D gets
-        // W in [288,352) and U' in [352,416)
-        const uint32_t hi = 16u << 16;
-        if (need_v) {
-          const uint32_t id = idesc_bf16_f32(64, 128, 0, 1);
-          umma_k_loop(tmem + TM_WU, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ, OFF_V - OFF_KQ, false, 0, 4, id, false);
-          umma_k_loop(tmem + TM_WU + hi, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ + 16384, OFF_V + 8192 - OFF_KQ - 16384,
-                      false, 0, 4, id, false);
-        } else {
-          const uint32_t id = idesc_bf16_f32(64, 64, 0, 1);
-          umma_k_loop(tmem + TM_WU, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ, 16384, false, 0, 4, id, false);
-          umma_k_loop(tmem + TM_WU + hi, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ + 16384, 16384, false, 0, 4, id,
-                      false);
-        }
-      }
-      if (tid == 0) umma_commit(&m->mma);
+      ops_arrive();  // ---------------------------------------------- UMMA: W = T' Kt, U' = T' V
       if (write_out && j > 0) epilogue_b(L_prev, tok_prev);  // in the shadow of the W|U' UMMAs
       {
         const bool r = wg_wait(&m->mma, mph & 1u);
@@ -859,20 +926,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           at16(sm, OFF_KL + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
         }
       }
-      sync_for_mma();
-      // ---------------------------------------------------------------- UMMA: U = U' - W S0 ; O = Qt S0
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t id = idesc_bf16_f32(64, 64, 0, 1);
-        const uint32_t hi = 16u << 16;
-        umma_k_loop(tmem + TM_WU + 64, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S, 16384, false, 0, 8, id, need_v);
-        umma_k_loop(tmem + TM_WU + 64 + hi, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S + 16384, 16384, false, 0, 8,
-                    id, need_v);
-        umma_k_loop(tmem + TM_O, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S, 16384, false, 0, 8, id, false);
-        umma_k_loop(tmem + TM_O + hi, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S + 16384, 16384, false, 0, 8,
-                    id, false);
-        umma_commit(&m->mma);
-      }
+      ops_arrive();  // ---------------------------------------------- UMMA: U = U' - W S0 ; O = Qt S0
       // in the shadow of these UMMAs (they read the bf16 copy of S, not TMEM columns [0,128)):
       // S <- Diag(e^{gamma_C}) S in TMEM, then the next chunk's decay scan, whose g tile the
       // producer fetched during this chunk; its release lets the producer fetch the one after
@@ -921,24 +975,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           at16(sm, OFF_KL + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
         }
       }
-      sync_for_mma();
-      // ---------------------------------------------------------------- UMMA: O += P U ; S += Kh^T U
-      if (tid == 0) {
+      ops_arrive();  // ---------------------------------------------- UMMA: O += P U ; S += Kh^T U
+      // in their shadow: stage this chunk's gate logits for its epilogue (the buffer's previous
+      // contents were consumed beside this chunk's W|U' UMMAs)
+      if (write_out) load_gate(L, tok);
+      {
+        const bool r = wg_wait(&m->mma, mph & 1u);
+        ++mph;
         tc_fence_after();
-        umma_k_loop(tmem + TM_O, sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL, 8192, false, 0, 4,
-                    idesc_bf16_f32(64, 64, 0, 1), true);
-        umma_k_loop(tmem + TM_O + (16u << 16), sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL + 8192, 8192, false, 0, 4,
-                    idesc_bf16_f32(64, 64, 0, 1), true);
-        umma_k_loop(tmem + TM_S, sm_u + OFF_KH, 8192, false, 0, sm_u + OFF_KL, 8192, false, 0, 4,
-                    idesc_bf16_f32(128, 128, 1, 1), true);
+        if (!r) { ok = false; break; }
       }
-      if (!mma_commit_wait()) { ok = false; break; }
 
       L_prev = L;
       tok_prev = tok;
     }
     if (ok && write_out && nchunks > 0) {
-      load_gate(L_prev, tok_prev);
       cp_async_wait_all();
       sync_wg();
       epilogue_a(L_prev, tok_prev);
@@ -975,10 +1026,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-    } else if (tid == 0 && mph > 0) {
-      // an aborted UMMA group may still be running: wait for it before freeing TMEM
-      wait_bounded(&m->mma, (mph - 1) & 1u, m, drain_limit, p.error_word, false);
     }
+    cp_async_wait_all();  // no gate copy may outlive the block (after an abort)
   }
   tc_fence_before();
   __syncthreads();
