@@ -168,24 +168,17 @@ __device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], 
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
-// fp32-accurate product from three tf32 MMAs: with x = x_hi + x_lo (both tf32), a b ~ a_hi b_hi
-// + a_hi b_lo + a_lo b_hi, each term into its own accumulator d[0..2] (three independent MMA
-// chains); the dropped a_lo b_lo is below fp32 rounding.
-__device__ __forceinline__ void mma_3xtf32(float (&d)[3][4], const float (&a)[4], const float (&b)[2]) {
-  uint32_t ah[4], al[4], bh[2], bl[2];
+// d += a b with both operands rounded to tf32 (nearest).  The inverse's off-diagonal blocks only
+// feed T' = T Diag(beta), which is rounded to bf16 (8 mantissa bits) for the W|U' UMMAs; tf32 (11
+// bits) products leave the output and state errors unchanged (checked against the oracle on the
+// chunk model).
+__device__ __forceinline__ void mma_1xtf32(float (&d)[4], const float (&a)[4], const float (&b)[2]) {
+  uint32_t ah[4], bh[2];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    ah[i] = tf32_rna(a[i]);
-    al[i] = tf32_rna(a[i] - __uint_as_float(ah[i]));
-  }
+  for (int i = 0; i < 4; ++i) ah[i] = tf32_rna(a[i]);
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    bh[i] = tf32_rna(b[i]);
-    bl[i] = tf32_rna(b[i] - __uint_as_float(bh[i]));
-  }
-  mma_tf32(d[0], ah, bh);
-  mma_tf32(d[1], ah, bl);
-  mma_tf32(d[2], al, bh);
+  for (int i = 0; i < 2; ++i) bh[i] = tf32_rna(b[i]);
+  mma_tf32(d, ah, bh);
 }
 
 // One accumulation chain of a UMMA group: destination, descriptors (built once), operand majors
@@ -819,7 +812,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Off-diagonal blocks level by level (block distance d), one 16x8 strip per warp: warp
         // w < 2 (4 - d) takes a = b + d with b = w / 2 and columns 16 b + 8 (w % 2) .. +7:
         //   Y = sum_{c=b}^{a-1} L_ac T_cb,   T_ab = -T_aa Y,
-        // as m16n8k8 3xTF32 MMAs.  Y never leaves the warp: its C fragment becomes the B fragment
+        // as m16n8k8 tf32 MMAs.  Y never leaves the warp: its C fragment becomes the B fragment
         // of the second product by shuffles.  A level reads only blocks of earlier levels.
         {
           const int g = lane >> 2, t4 = lane & 3;
@@ -827,13 +820,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int d = 1; d <= 3; ++d) {
             if (warp < 2 * (4 - d)) {
               const int b = warp >> 1, n0 = 8 * (warp & 1), a = b + d;
-              float acc[2][3][4];  // by K-step parity and 3xTF32 term: six independent chains
+              float acc[2][4];  // by K-step parity: two independent chains
 #pragma unroll
               for (int u = 0; u < 2; ++u)
 #pragma unroll
-                for (int v = 0; v < 3; ++v)
-#pragma unroll
-                  for (int i = 0; i < 4; ++i) acc[u][v][i] = 0.f;
+                for (int i = 0; i < 4; ++i) acc[u][i] = 0.f;
               const float* la = Lf + (16 * a + g) * LDF + t4;
               const float* tb = Tf + t4 * LDT + 16 * b + n0 + g;
 #pragma unroll
@@ -841,12 +832,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int kk = 16 * b + 8 * ks;
                 const float af[4] = {la[kk], la[8 * LDF + kk], la[kk + 4], la[8 * LDF + kk + 4]};
                 const float bf[2] = {tb[kk * LDT], tb[(kk + 4) * LDT]};
-                mma_3xtf32(acc[ks & 1], af, bf);
+                mma_1xtf32(acc[ks & 1], af, bf);
               }
               float y[4];
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                y[i] = (acc[0][0][i] + acc[1][0][i]) + ((acc[0][1][i] + acc[1][1][i]) + (acc[0][2][i] + acc[1][2][i]));
+              for (int i = 0; i < 4; ++i) y[i] = acc[0][i] + acc[1][i];
               // Y[r][n] sits in lane 4 (r % 8) + n / 2, register 2 (r / 8) + n % 2; this lane needs
               // Y[t][g], Y[t+4][g] (first K step) and Y[8+t][g], Y[12+t][g] (second)
               const int s0 = 4 * t4 + (g >> 1), s1 = s0 + 16;
@@ -859,24 +849,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float u3 = __shfl_sync(0xffffffffu, y[2], s1), v3 = __shfl_sync(0xffffffffu, y[3], s1);
                 yb[0] = odd ? v0 : u0; yb[1] = odd ? v1 : u1; yb[2] = odd ? v2 : u2; yb[3] = odd ? v3 : u3;
               }
-              float oacc[2][3][4];
+              float oacc[2][4];
 #pragma unroll
               for (int u = 0; u < 2; ++u)
 #pragma unroll
-                for (int v = 0; v < 3; ++v)
-#pragma unroll
-                  for (int i = 0; i < 4; ++i) oacc[u][v][i] = 0.f;
+                for (int i = 0; i < 4; ++i) oacc[u][i] = 0.f;
               const float* ta = Tf + (16 * a + g) * LDT + 16 * a + t4;
 #pragma unroll
               for (int ks = 0; ks < 2; ++ks) {
                 const float af[4] = {-ta[8 * ks], -ta[8 * LDT + 8 * ks], -ta[8 * ks + 4], -ta[8 * LDT + 8 * ks + 4]};
                 const float bf[2] = {yb[2 * ks], yb[2 * ks + 1]};
-                mma_3xtf32(oacc[ks], af, bf);
+                mma_1xtf32(oacc[ks], af, bf);
               }
               float o4[4];
 #pragma unroll
-              for (int i = 0; i < 4; ++i)
-                o4[i] = (oacc[0][0][i] + oacc[1][0][i]) + ((oacc[0][1][i] + oacc[1][1][i]) + (oacc[0][2][i] + oacc[1][2][i]));
+              for (int i = 0; i < 4; ++i) o4[i] = oacc[0][i] + oacc[1][i];
               float* to = Tf + (16 * a + g) * LDT + 16 * b + n0 + 2 * t4;
               *reinterpret_cast<float2*>(to) = make_float2(o4[0], o4[1]);
               *reinterpret_cast<float2*>(to + 8 * LDT) = make_float2(o4[2], o4[3]);
