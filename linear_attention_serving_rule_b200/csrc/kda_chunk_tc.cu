@@ -90,7 +90,9 @@ __host__ __device__ constexpr uint32_t ap_off(int a) { return a == 0 ? 0u : a ==
 constexpr uint32_t KC_ROWS = 160, KC_BLK = KC_ROWS * 128;
 
 struct Misc {
-  uint64_t full_g, full_kq, full_v, empty_g, empty_kq, empty_v, mma, ops;
+  // k and q have their own barriers: the k rows are free after the W|U' UMMAs, the q rows only
+  // after the U/O UMMAs
+  uint64_t full_g, full_k, full_q, full_v, empty_g, empty_k, empty_q, empty_v, mma, ops;
   uint32_t tmem_base;
   int32_t abort;
   float beta[2][C];  // double-buffered by chunk parity (written by the producer warp)
@@ -240,8 +242,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool need_v = seg.role != kRoleLocalM;  // the transition pass runs with values = 0
 
   if (tid == 0) {
-    mbar_init(&m->full_g, 1); mbar_init(&m->full_kq, 1); mbar_init(&m->full_v, 1);
-    mbar_init(&m->empty_g, 1); mbar_init(&m->empty_kq, 1); mbar_init(&m->empty_v, 1);
+    mbar_init(&m->full_g, 1); mbar_init(&m->full_k, 1); mbar_init(&m->full_q, 1); mbar_init(&m->full_v, 1);
+    mbar_init(&m->empty_g, 1); mbar_init(&m->empty_k, 1); mbar_init(&m->empty_q, 1); mbar_init(&m->empty_v, 1);
     mbar_init(&m->mma, 1);
     mbar_init(&m->ops, 8);  // one arrival per compute warp: a UMMA group's operands are in place
     m->abort = 0;
@@ -264,11 +266,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ===================================================================== TMA producer
     // Lane 0 issues the tile loads; the whole warp first fetches the chunk's beta into the
     // double buffer m->beta[j & 1], published by the same mbarrier as the g tile.
-    int ig = -1, ikq = -1, iv = -1;  // last chunk whose g, k|q and v loads were issued
+    int ig = -1, ik = -1, iq = -1, iv = -1;  // last chunk whose g, k, q and v loads were issued
     for (int j = 0; j < nchunks; ++j) {
       const int32_t tok = seg.tok0 + j * C;
       const int L = min(C, seg.len - j * C);
       const uint32_t par = (uint32_t)((j & 1) ^ 1);
+      // the chunk's k, q and v tiles into L2 now, about a chunk before their buffers free up (the q
+      // load is issued only once the previous chunk's U/O UMMAs are done, on the critical path)
+      if (lane == 0) {
+        for (int hf = 0; hf < 2; ++hf) {
+          tma_prefetch_3d(&maps.k, hf * 64, h, tok);
+          tma_prefetch_3d(&maps.q, hf * 64, h, tok);
+          if (need_v) tma_prefetch_3d(&maps.v, hf * 64, h, tok);
+        }
+      }
       int okw = 1;
       if (lane == 0) okw = wait_bounded(&m->empty_g, par, m, drain_limit, p.error_word) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);
@@ -286,17 +297,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hf = 0; hf < 2; ++hf) tma_load_3d(sm + OFF_G + hf * 8192, &maps.g, &m->full_g, hf * 64, h, tok);
       }
       ig = j;
-      if (lane == 0) okw = wait_bounded(&m->empty_kq, par, m, drain_limit, p.error_word) ? 1 : 0;
+      if (lane == 0) okw = wait_bounded(&m->empty_k, par, m, drain_limit, p.error_word) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);
       if (!okw) break;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&m->full_kq, 2 * 16384);
-        for (int hf = 0; hf < 2; ++hf) {
-          tma_load_3d(sm + OFF_KQ + hf * 16384, &maps.k, &m->full_kq, hf * 64, h, tok);
-          tma_load_3d(sm + OFF_KQ + hf * 16384 + 8192, &maps.q, &m->full_kq, hf * 64, h, tok);
-        }
+        mbar_arrive_expect_tx(&m->full_k, 16384);
+        for (int hf = 0; hf < 2; ++hf) tma_load_3d(sm + OFF_KQ + hf * 16384, &maps.k, &m->full_k, hf * 64, h, tok);
       }
-      ikq = j;
+      ik = j;
+      if (lane == 0) okw = wait_bounded(&m->empty_q, par, m, drain_limit, p.error_word) ? 1 : 0;
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (!okw) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&m->full_q, 16384);
+        for (int hf = 0; hf < 2; ++hf)
+          tma_load_3d(sm + OFF_KQ + hf * 16384 + 8192, &maps.q, &m->full_q, hf * 64, h, tok);
+      }
+      iq = j;
       if (!need_v) continue;
       if (lane == 0) okw = wait_bounded(&m->empty_v, par, m, drain_limit, p.error_word) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);
@@ -310,7 +327,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // drain: after an abort, wait (bounded, regardless of the abort) for the loads issued
     if (lane == 0 && *(volatile int32_t*)&m->abort) {
       if (ig >= 0) wait_bounded(&m->full_g, (uint32_t)(ig & 1), m, drain_limit, p.error_word, false);
-      if (ikq >= 0) wait_bounded(&m->full_kq, (uint32_t)(ikq & 1), m, drain_limit, p.error_word, false);
+      if (ik >= 0) wait_bounded(&m->full_k, (uint32_t)(ik & 1), m, drain_limit, p.error_word, false);
+      if (iq >= 0) wait_bounded(&m->full_q, (uint32_t)(iq & 1), m, drain_limit, p.error_word, false);
       if (iv >= 0) wait_bounded(&m->full_v, (uint32_t)(iv & 1), m, drain_limit, p.error_word, false);
     }
   } else if (warp == 9) {
@@ -626,7 +644,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* beta = m->beta[j & 1];
       // ---------------------------------------------------------------- decay prep: all bf16 operands
 
-      if (!wg_wait(&m->full_kq, par)) { ok = false; break; }
+      {
+        if (tid == 0 && wait_bounded(&m->full_k, par, m, limit, p.error_word))
+          wait_bounded(&m->full_q, par, m, limit, p.error_word);
+        sync_wg();
+        if (*(volatile int32_t*)&m->abort != 0) { ok = false; break; }
+      }
       if (l2norm) {  // sums of squares of the raw k | q rows (two column halves per row)
         const int rr = tid & 127, hf = tid >> 7;
         float ss = 0.f;
@@ -895,7 +918,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (!r) { ok = false; break; }
       }
-      if (tid == 0 && need_v) mbar_arrive(&m->empty_v);
+      if (tid == 0) {  // v and the k rows (e^{gamma} k in place) consumed
+        if (need_v) mbar_arrive(&m->empty_v);
+        mbar_arrive(&m->empty_k);
+      }
 
       // ---------------------------------------------------------------- -W -> bf16
       // lane l < 16: row 16 q + l, columns 32 wg ..; lane l + 16: the same row, columns 64 + 32 wg ..
@@ -945,7 +971,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (!r || !next_ok) { ok = false; break; }
       }
-      if (tid == 0) mbar_arrive(&m->empty_kq);  // k, q and their in-place products consumed
+      if (tid == 0) mbar_arrive(&m->empty_q);  // the q rows (e^{gamma} q in place) consumed
 
       // ---------------------------------------------------------------- U -> bf16 (same lane split as -W)
       {
