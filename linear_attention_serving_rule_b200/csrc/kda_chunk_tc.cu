@@ -149,6 +149,21 @@ __device__ __forceinline__ void unpack8(uint4 u, float (&f)[8]) {
 __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
   return make_uint4(f2_to_bf2(f[0], f[1]), f2_to_bf2(f[2], f[3]), f2_to_bf2(f[4], f[5]), f2_to_bf2(f[6], f[7]));
 }
+// The same 8 values as 4 pairs, for the two-wide fp32 multiply (mul.rn.f32x2: each half rounds
+// like mul.rn.f32, so results match the scalar products bit for bit).
+__device__ __forceinline__ void unpack8x2(uint4 u, float2 (&f)[4]) {
+  f[0] = bf2_to_f2(u.x); f[1] = bf2_to_f2(u.y); f[2] = bf2_to_f2(u.z); f[3] = bf2_to_f2(u.w);
+}
+__device__ __forceinline__ uint4 pack8x2(const float2 (&f)[4]) {
+  return make_uint4(f2_to_bf2(f[0].x, f[0].y), f2_to_bf2(f[1].x, f[1].y), f2_to_bf2(f[2].x, f[2].y),
+                    f2_to_bf2(f[3].x, f[3].y));
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(*reinterpret_cast<const uint64_t*>(&a)),
+      "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<const float2*>(&r);
+}
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -685,61 +700,73 @@ __global__ void __launch_bounds__(kThreads, 1)
           s2[e] = b == 0 ? se[2] : b == 1 ? se[3] : 1.f;
           s3[e] = se[3];
         }
+        float2 Eb2[4], sb2[4], s1_2[4], s2_2[4], s3_2[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          Eb2[c] = make_float2(Eb[2 * c], Eb[2 * c + 1]);
+          sb2[c] = make_float2(sb[2 * c], sb[2 * c + 1]);
+          s1_2[c] = make_float2(s1[2 * c], s1[2 * c + 1]);
+          s2_2[c] = make_float2(s2[2 * c], s2[2 * c + 1]);
+          s3_2[c] = make_float2(s3[2 * c], s3[2 * c + 1]);
+        }
+        // channel pairs (2c, 2c+1) as float2 throughout
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int t = t0 + i;
-          float kf[8], qf[8], x[8], ix[8], f[8];
+          float2 kf[4], qf[4], x[4], ix[4], f[4], fq[4];
           if (t < L) {
-            unpack8(at16(sm, OFF_KQ + sw128_oct(t, o, 16384)), kf);
-            unpack8(at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)), qf);
+            unpack8x2(at16(sm, OFF_KQ + sw128_oct(t, o, 16384)), kf);
+            unpack8x2(at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)), qf);
             if (l2norm) {  // x / sqrt(|x|^2 + eps)
               const float rk = rsqrtf(m->qkss[0][t] + m->qkss[1][t] + KDA_L2NORM_EPS);
               const float rq = rsqrtf(m->qkss[0][64 + t] + m->qkss[1][64 + t] + KDA_L2NORM_EPS);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) { kf[e] *= rk; qf[e] *= rq; }
+              for (int c = 0; c < 4; ++c) {
+                kf[c] = fmul2(kf[c], make_float2(rk, rk));
+                qf[c] = fmul2(qf[c], make_float2(rq, rq));
+              }
             }
           } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) { kf[e] = 0.f; qf[e] = 0.f; }
+            for (int c = 0; c < 4; ++c) { kf[c] = make_float2(0.f, 0.f); qf[c] = make_float2(0.f, 0.f); }
           }
 #pragma unroll
-          for (int e = 0; e < 8; ++e) { x[e] = ex2(gl[i][e]); ix[e] = ex2(-gl[i][e]); }
+          for (int c = 0; c < 4; ++c) {
+            x[c] = make_float2(ex2(gl[i][2 * c]), ex2(gl[i][2 * c + 1]));
+            ix[c] = make_float2(ex2(-gl[i][2 * c]), ex2(-gl[i][2 * c + 1]));
+          }
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = kf[e] * x[e];
-          at16(sm, OFF_KL + sw128_oct(t, o, 16384)) = pack8(f);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = qf[e] * x[e];
-          at16(sm, OFF_KL + sw128_oct(64 + t, o, 16384)) = pack8(f);
+          for (int c = 0; c < 4; ++c) { f[c] = fmul2(kf[c], x[c]); fq[c] = fmul2(qf[c], x[c]); }
+          at16(sm, OFF_KL + sw128_oct(t, o, 16384)) = pack8x2(f);
+          at16(sm, OFF_KL + sw128_oct(64 + t, o, 16384)) = pack8x2(fq);
           // e^{gamma} k and e^{gamma} q, in place over the raw tiles (this thread's own elements)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = kf[e] * x[e] * Eb[e];
-          at16(sm, OFF_KQ + sw128_oct(t, o, 16384)) = pack8(f);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = qf[e] * x[e] * Eb[e];
-          at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)) = pack8(f);
+          for (int c = 0; c < 4; ++c) { f[c] = fmul2(f[c], Eb2[c]); fq[c] = fmul2(fq[c], Eb2[c]); }
+          at16(sm, OFF_KQ + sw128_oct(t, o, 16384)) = pack8x2(f);
+          at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)) = pack8x2(fq);
           // Kc_a = k e^{r_a - gamma_t}: k ix for a = b, then k ix se_b se_{b+1} ... se_{a-1};
           // the last one (a = 3) times se_3 is e^{gamma_C - gamma_t} k, the state-carry operand
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] = kf[e] * ix[e];
-          at16(sm, OFF_KC + sw128_oct(ap_off(b) + t, o, KC_BLK)) = pack8(f);
+          for (int c = 0; c < 4; ++c) f[c] = fmul2(kf[c], ix[c]);
+          at16(sm, OFF_KC + sw128_oct(ap_off(b) + t, o, KC_BLK)) = pack8x2(f);
           if (b < 3) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) f[e] = kf[e] * ix[e] * sb[e];
-            at16(sm, OFF_KC + sw128_oct(ap_off(b + 1) + t, o, KC_BLK)) = pack8(f);
+            for (int c = 0; c < 4; ++c) f[c] = fmul2(f[c], sb2[c]);
+            at16(sm, OFF_KC + sw128_oct(ap_off(b + 1) + t, o, KC_BLK)) = pack8x2(f);
             if (b < 2) {
 #pragma unroll
-              for (int e = 0; e < 8; ++e) f[e] *= s1[e];
-              at16(sm, OFF_KC + sw128_oct(ap_off(b + 2) + t, o, KC_BLK)) = pack8(f);
+              for (int c = 0; c < 4; ++c) f[c] = fmul2(f[c], s1_2[c]);
+              at16(sm, OFF_KC + sw128_oct(ap_off(b + 2) + t, o, KC_BLK)) = pack8x2(f);
               if (b < 1) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] *= s2[e];
-                at16(sm, OFF_KC + sw128_oct(ap_off(3) + t, o, KC_BLK)) = pack8(f);
+                for (int c = 0; c < 4; ++c) f[c] = fmul2(f[c], s2_2[c]);
+                at16(sm, OFF_KC + sw128_oct(ap_off(3) + t, o, KC_BLK)) = pack8x2(f);
               }
             }
           }
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] *= s3[e];
-          at16(sm, OFF_KH + sw128_oct(t, o, 8192)) = pack8(f);
+          for (int c = 0; c < 4; ++c) f[c] = fmul2(f[c], s3_2[c]);
+          at16(sm, OFF_KH + sw128_oct(t, o, 8192)) = pack8x2(f);
         }
       }
       if (tid < DK) {
