@@ -36,10 +36,16 @@ struct DecodeParams {
   void* out;
   float* position_states;  // [N, K, H, dk, dv] or null
   int32_t H, num_slots, tokens;
+  int32_t ahead;  // CTAs resident at once: the unit this many ahead gets its state prefetched
   float scale, eps;
   uint32_t flags;
   uint32_t* error_word;
 };
+
+// Bulk prefetch of [addr, addr + bytes) into L2 (a hint: no completion, no shared memory).
+__device__ __forceinline__ void prefetch_l2(const void* addr, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(addr), "r"(bytes) : "memory");
+}
 
 // kPre: the pre-processing of the raw projections (KDA_FLAG_G_LOGITS, KDA_FLAG_BETA_LOGITS,
 // KDA_FLAG_QK_L2NORM) is compiled in; the instance without it is the plain step.
@@ -79,6 +85,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
 #pragma unroll
   for (int i = 0; i < NP; ++i)
     s[i] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)(r0 + RPP * i) * DV) + cg);
+  // CTAs start in index order as earlier ones retire, so the unit `ahead` places on is likely to
+  // start about when this one ends: pull its state into L2 now, keeping HBM busy across the gap
+  // between one CTA's stores and the next one's loads
+  if (tid == 0 && p.ahead > 0 && unit + p.ahead < (int)gridDim.x) {
+    const int u2 = unit + p.ahead;
+    const int n2 = u2 / p.H;
+    const int slot2 = p.state_indices ? p.state_indices[n2] : n2;
+    if (slot2 >= 0 && slot2 < p.num_slots)
+      prefetch_l2(p.state + ((size_t)slot2 * p.H + (u2 - n2 * p.H)) * (size_t)(DK * DV),
+                  (uint32_t)(DK * DV * sizeof(float)));
+  }
 
   const int K = p.tokens;
   const bool commit = (p.flags & KDA_FLAG_DECODE_NO_COMMIT) == 0;
@@ -196,13 +213,35 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   }
 }
 
+// CTAs of one kernel instance resident on the whole device at once (cached per device)
+template <typename T, int DK, int DV, bool kPre>
+int resident_ctas() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int per_sm = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<T, DK, DV, kPre>, kThreads, 0) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return 0;
+    cache[dev] = per_sm * sms > 0 ? per_sm * sms : -1;
+  }
+  return cache[dev] > 0 ? cache[dev] : 0;
+}
+
+template <typename T, int DK, int DV, bool kPre>
+cudaError_t launch_pre(DecodeParams p, int units, cudaStream_t stream) {
+  p.ahead = resident_ctas<T, DK, DV, kPre>();
+  decode_kernel<T, DK, DV, kPre><<<units, kThreads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
 template <typename T, int DK, int DV>
 cudaError_t launch_t(const DecodeParams& p, int units, cudaStream_t stream) {
   if (p.flags & (KDA_FLAG_G_LOGITS | KDA_FLAG_BETA_LOGITS | KDA_FLAG_QK_L2NORM))
-    decode_kernel<T, DK, DV, true><<<units, kThreads, 0, stream>>>(p);
-  else
-    decode_kernel<T, DK, DV, false><<<units, kThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+    return launch_pre<T, DK, DV, true>(p, units, stream);
+  return launch_pre<T, DK, DV, false>(p, units, stream);
 }
 
 template <typename T>
@@ -224,6 +263,7 @@ cudaError_t launch_decode(const kda_decode_args& a, cudaStream_t stream) {
   p.out = a.out;
   p.position_states = a.position_states;
   p.tokens = a.tokens > 0 ? a.tokens : 1;
+  p.ahead = 0;
   p.H = a.H;
   p.num_slots = a.num_slots;
   p.scale = a.scale;
