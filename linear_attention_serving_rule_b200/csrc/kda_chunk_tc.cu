@@ -21,9 +21,11 @@
 // operand Kc_a = k e^{r_a - gamma} over the first 16(a+1) tokens; one M=128 UMMA per a
 // produces A (rows 0-63) and P (rows 64-127) from the stacked operand [k; q] e^{gamma - r_own}.
 //
-// Work split (320 threads): warp 8 is the TMA producer with three groups of tiles: g (with beta,
-// handed back right after the decay scan), k and q (landing interleaved as one 128-row tile;
-// handed back after the UMMAs that read their in-place products) and v (after W/U').  Warps 0-7
+// Work split (320 threads): warp 8 is the TMA producer with four groups of tiles: g (with beta,
+// handed back right after the decay scan), k and q (landing interleaved as one 128-row tile, each
+// with its own barrier: k is handed back after the W|U' UMMAs, q after the U/O UMMAs that read
+// its in-place product) and v (after W|U'); it also prefetches each chunk's k, q and v tiles into
+// L2 about a chunk ahead.  Warps 0-7
 // are two compute warpgroups; warp w owns TMEM lane quarter w % 4.  Decay prep, Gram read-out,
 // UT inverse and the -W / U conversions run on all 256 threads; in the shadow of the Gram and of
 // the W|U' UMMAs both warpgroups run the previous chunk's epilogue; while warps 0-1 invert the
