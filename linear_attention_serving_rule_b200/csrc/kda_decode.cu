@@ -223,8 +223,10 @@ int resident_ctas() {
     int per_sm = 0, sms = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<T, DK, DV, kPre>, kThreads, 0) !=
             cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      (void)cudaGetLastError();  // no prefetch then; the launch's own error check must not see this
       return 0;
+    }
     cache[dev] = per_sm * sms > 0 ? per_sm * sms : -1;
   }
   return cache[dev] > 0 ? cache[dev] : 0;
