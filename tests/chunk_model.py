@@ -47,10 +47,13 @@ def _ident(x):
     return x
 
 
-def chunk_unit(q, k, v, g, beta, S0, *, C=64, sub=16, scale=None, rnd=None, state_rnd=None):
+def chunk_unit(q, k, v, g, beta, S0, *, C=64, sub=16, scale=None, rnd=None, state_rnd=None, stacked=False):
     """One unit: q, k, g [T, dk]; v [T, dv]; beta [T]; S0 [dk, dv].  fp64 arithmetic.
     rnd: rounding applied to bf16 operands (None = exact); state_rnd: rounding of the
-    state copy used as an MMA operand (defaults to rnd)."""
+    state copy used as an MMA operand (defaults to rnd).
+    stacked: the output through the stacked operands [T'; P T'] and [-W; Q~ - P W] (U and the
+    whole O from one product with S, no separate P U term), with that form's own rounding
+    points: P T' and Q~ - P W are rounded like the other bf16 operands, P U' stays fp32."""
     q, k, v, g, beta = (np.asarray(a, dtype=np.float64) for a in (q, k, v, g, beta))
     T, dk = q.shape
     dv = v.shape[1]
@@ -91,7 +94,11 @@ def chunk_unit(q, k, v, g, beta, S0, *, C=64, sub=16, scale=None, rnd=None, stat
         Sb = RS(S)
         U = Up - R(W) @ Sb
         Ub = R(U)
-        O = scale * (Qt @ Sb + R(P) @ Ub)
+        if stacked:
+            PT = R(R(P) @ Tp)                            # second half of the stacked T' operand
+            O = scale * (PT @ V + R(Qt - PT @ Kt) @ Sb)  # = scale (Q~ S + P U) in exact arithmetic
+        else:
+            O = scale * (Qt @ Sb + R(P) @ Ub)
         Kh = R(K * np.exp(gam[C - 1] - gam))             # e^{gamma_C - gamma} k
         S = np.exp(gam[C - 1])[:, None] * S + Kh.T @ Ub
         out[c0:c0 + L] = O[:L]

@@ -55,3 +55,23 @@ def test_bf16_operand_error_budget(decay_shift):
     o, f = cm.chunk_forward(a["q"], a["k"], a["v"], a["g"], a["beta"], cu, S0=s0, C=64, rnd=cm.bf16)
     assert _rel(o, o_ref) < 5e-3
     assert _rel(f, f_ref) < 3.5e-3
+
+
+def test_stacked_output_form_equals_oracle_and_keeps_the_budget():
+    """O = Q~ S + P U rewritten as P T' V + (Q~ - P T' K~) S (the operands [T'; P T'] and
+    [-W; Q~ - P W] stacked over 128 rows): exact to rounding, and inside the same bf16 error
+    budget as the form the kernel uses now."""
+    a, s0, cu = _inputs([1, 15, 16, 17, 63, 64, 65, 150], 32, 24, seed=24)
+    o_ref, f_ref = oracle.forward(a["q"], a["k"], a["v"], a["g"], a["beta"], cu_seqlens=cu,
+                                  initial_state=s0)
+    o, f = cm.chunk_forward(a["q"], a["k"], a["v"], a["g"], a["beta"], cu, S0=s0, C=64, stacked=True)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(f, f_ref, rtol=1e-10, atol=1e-12)
+    for shift in (0.0, -6.0):
+        a, s0, cu = _inputs([300, 211], 128, 128, seed=23, dtype="bf16", decay_shift=shift)
+        o_ref, f_ref = oracle.forward(a["q"], a["k"], a["v"], a["g"], a["beta"], cu_seqlens=cu,
+                                      initial_state=s0)
+        o, f = cm.chunk_forward(a["q"], a["k"], a["v"], a["g"], a["beta"], cu, S0=s0, C=64, rnd=cm.bf16,
+                                stacked=True)
+        assert _rel(o, o_ref) < 5e-3, shift
+        assert _rel(f, f_ref) < 3.5e-3, shift
