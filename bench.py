@@ -60,6 +60,10 @@ def parse_args():
     ap.add_argument("--no-snapshots", action="store_true")
     ap.add_argument("--no-preprocess", action="store_true")
     ap.add_argument("--no-unbounded", action="store_true")
+    ap.add_argument("--no-varlen", action="store_true")
+    ap.add_argument("--no-long", action="store_true")
+    ap.add_argument("--long-tokens", type=int, default=1 << 20,
+                    help="tokens of the long-context sequence (default 2^20, the full workload)")
     return ap.parse_args()
 
 
@@ -285,7 +289,9 @@ def run_ours(args):
     ws_bytes = kda.kda_chunk_fwd_workspace_size(a)
     ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
     a.workspace, a.workspace_bytes = ws.data_ptr(), ws_bytes
-    launches_per_call = 1  # 128 units fill the GPU: no split, one kernel per call
+    # 128 (sequence, head) units on 148 SMs: the automatic split only cuts sequences when the units
+    # fill less than half the GPU, so this batch runs as one kernel per call
+    launches_per_call = 1
     input_bytes = sum(t.numel() * t.element_size() for t in (inp.q, inp.k, inp.v, inp.g, inp.beta, inp.gate))
 
     def call():
@@ -360,6 +366,15 @@ def run_ours(args):
     if not args.no_decode:
         decode = run_decode(args, dev, stream, rank, world, peaks, peak_src, clocks)
         decode_multi = run_decode_multi(args, dev, stream, rank, peaks, decode["roofline"]["kernel_ms"])
+
+    # ---------------- the varlen and long-context prefill workloads (their own legs)
+    cpu_ok = rank == 0 and world == 1 and not args.no_cpu_baseline
+    varlen = None
+    if not args.no_varlen:
+        varlen = run_varlen(args, L, stream, dev, rank, world, peaks, peak_src, cpu_ok)
+    longctx = None
+    if not args.no_long:
+        longctx = run_long(args, L, stream, dev, rank, world, peaks, peak_src, cpu_ok)
     clocks.stop()
     clk = clocks.summary()
 
@@ -389,7 +404,7 @@ def run_ours(args):
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": launches_per_call * args.steps, "clocks": clk, "decode": decode,
             "snapshots": snaps, "preprocess": prep, "decode_multi": decode_multi,
-            "unbounded_decay": unb}
+            "unbounded_decay": unb, "varlen": varlen, "long_context": longctx}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -565,7 +580,11 @@ def run_decode(args, dev, stream, rank, world, peaks, peak_src, clocks):
     state_bytes = 2 * N * H * dk * dv * 4
     achieved = state_bytes / (kern_ms / 1e3) / 1e9
     traffic, sha = kernel_traffic("decode_bf16", ["linear_attention_serving_rule_b200/csrc/kda_decode.cu"])
-    return {"metric": "decode-step state HBM GB/s", "workload": f"decode bf16 N{N} x H{H} dk=dv={dk}, "
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = decode_cpu_baseline(state, toks, N, H, dk, dv, ring)
+    return {"metric": "decode-step state HBM GB/s", "cpu_baseline": cpu,
+            "workload": f"decode bf16 N{N} x H{H} dk=dv={dk}, "
             f"fp32 states in place, {steps} steps, ring of {ring} input sets",
             "value": world * state_bytes * steps / (ms / 1e3) / 1e9, "unit": "GB/s",
             "ms_per_step": ms / steps, "tokens_per_s": world * N * steps / (ms / 1e3),
@@ -574,6 +593,148 @@ def run_decode(args, dev, stream, rank, world, peaks, peak_src, clocks):
                          "alg_bytes_per_launch": state_bytes, "kernel_ms": kern_ms,
                          "kernel_source_sha1": sha},
             "gpu_launches": steps}
+
+
+def decode_cpu_baseline(state, toks, N, H, dk, dv, ring, n_seq=64, steps=16):
+    """The fp64 oracle's decode step on a sample of the batch (n_seq sequences, all heads, `steps`
+    consecutive steps over the same input ring), on the host cores: state GB/s in the GPU metric's
+    unit (fp32 state bytes read + written per step) and tokens/s."""
+    import numpy as np
+    import oracle
+    oracle.build()
+    cores = oracle.max_threads()
+    s64 = state[:n_seq].double().cpu().numpy()
+    h = lambda t: t.float().cpu().numpy()
+    sub = [{n: h(getattr(t, n)[:n_seq]) for n in ("q", "k", "v", "g", "beta", "gate")} for t in toks]
+    t0 = time.perf_counter()
+    for i in range(steps):
+        a = sub[i % ring]
+        oracle.decode_step(a["q"], a["k"], a["v"], a["g"], a["beta"], s64, gate=a["gate"])
+    dt = time.perf_counter() - t0
+    state_bytes = 2 * n_seq * H * dk * dv * 4 * steps
+    return {"value": state_bytes / dt / 1e9, "unit": "GB/s", "tokens_per_s": n_seq * steps / dt,
+            "cores": cores, "kind": "oracle",
+            "sample": f"{n_seq} sequences x H{H} (all heads) x {steps} consecutive steps of this decode "
+                      f"batch ({dt:.1f} s), fp64, OpenMP over (sequence, head) units"}
+
+
+def _time_calls(call, n, warmup, stream, dev):
+    """Mean CUDA-event time of `call` (ms) on `stream` after `warmup` untimed calls."""
+    import torch
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        ev[i][0].record(stream)
+        call()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    return statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+
+
+def _prefill_leg(args, L, stream, dev, world, peaks, peak_src, inp, H, n_calls, warmup, label,
+                 state_io_units, state_io_count):
+    """Time kda_chunk_fwd on `inp` (inputs resident in HBM): tokens/s and the HBM roofline on the
+    algorithmic bytes (1,538 B per head-token plus the fp32 states read and written)."""
+    import torch
+    import linear_attention_serving_rule_b200 as kda
+    from linear_attention_serving_rule_b200 import binding as B
+    out = torch.empty_like(inp.v)
+    N = inp.num_seqs
+    fin = torch.empty((N, H, 128, 128), dtype=torch.float32, device=dev)
+    a, keep = kda.make_chunk_args(inp.q, inp.k, inp.v, inp.g, inp.beta, gate=inp.gate,
+                                  cu_seqlens=inp.cu_seqlens, initial_state=inp.initial_state,
+                                  out=out, final_state=fin)
+    nb = kda.kda_chunk_fwd_workspace_size(a)
+    ws = torch.zeros(nb, dtype=torch.uint8, device=dev)
+    a.workspace, a.workspace_bytes = ws.data_ptr(), nb
+    sptr = stream.cuda_stream
+
+    def call():
+        rc = L.kda_chunk_fwd(ctypes.byref(a), sptr)
+        if rc != 0:
+            raise B.KdaError(rc, "kda_chunk_fwd")
+    barrier(world)
+    ms = _time_calls(call, n_calls, warmup, stream, dev)
+    ms = max_over_ranks(ms, world, dev)
+    st = kda.kda_read_device_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error in the {label} leg: {kda.kda_status_string(st)}")
+    del keep
+    tokens = inp.total_tokens
+    head_tokens = tokens * H
+    alg_bytes = head_tokens * BYTES_PER_HEAD_TOKEN + state_io_count * state_io_units * STATE_BYTES
+    achieved = alg_bytes / (ms / 1e3) / 1e9
+    tc = head_tokens * FLOPS_PER_HEAD_TOKEN / (ms / 1e3) / 1e12
+    return {"value": world * tokens / (ms / 1e3), "unit": UNIT, "tokens_per_call": tokens,
+            "head_tokens": head_tokens, "calls": n_calls, "kernel_ms": ms, "workspace_bytes": nb,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "peak_source": peak_src,
+                         "alg_bytes_per_call": alg_bytes,
+                         "tc_util": {"useful_tflops": tc, "frac": tc / peaks["bf16_tflops"]}}}
+
+
+def run_varlen(args, L, stream, dev, rank, world, peaks, peak_src, cpu_ok):
+    """64 packed sequences of U[128, 8192] tokens, H32, fp32 initial states read and final states
+    written: one kda_chunk_fwd call per step."""
+    import numpy as np
+    import torch
+    from linear_attention_serving_rule_b200 import synth
+    w = synth.WORKLOADS["varlen_bf16"]
+    inp = synth.make_workload("varlen_bf16", device=dev, seed=rank_seed(w["seed"], rank))
+    H = w["H"]
+    N = inp.num_seqs
+    res = _prefill_leg(args, L, stream, dev, world, peaks, peak_src, inp, H, n_calls=10, warmup=3,
+                       label="varlen", state_io_units=N * H, state_io_count=2)
+    lens = np.diff(inp.cu_seqlens)
+    res["workload"] = (f"KDA varlen packed prefill bf16: {N} sequences, lengths U[128, 8192] "
+                       f"({int(lens.min())}..{int(lens.max())}, {inp.total_tokens} tokens), H{H} d128, "
+                       f"gate + RMSNorm, fp32 initial and final states")
+    if cpu_ok:
+        import oracle
+        oracle.build()
+        cores = oracle.max_threads()
+        rng = np.random.default_rng(5)
+        units = [(int(n), int(h)) for n, h in zip(rng.integers(N, size=2 * cores), rng.integers(H, size=2 * cores))]
+        r, dt, ht = oracle_sample_tokens_per_s(inp, H, units)
+        res["cpu_baseline"] = {"value": r, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": f"{len(units)} random (sequence, head) units of this batch "
+                                         f"({ht} head-tokens, {dt:.1f} s), fp64, OpenMP over units"}
+    del inp
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_long(args, L, stream, dev, rank, world, peaks, peak_src, cpu_ok):
+    """One 2^20-token sequence, H16: 16 units for 148 SMs, so the library splits the sequence
+    (pass 1 per segment, the combine, pass 2); one kda_chunk_fwd call per step."""
+    import numpy as np
+    import torch
+    from linear_attention_serving_rule_b200 import synth
+    w = synth.WORKLOADS["long_bf16"]
+    T = int(args.long_tokens)
+    inp = synth.make_workload("long_bf16", device=dev, seed=rank_seed(w["seed"], rank), T=T)
+    H = w["H"]
+    res = _prefill_leg(args, L, stream, dev, world, peaks, peak_src, inp, H, n_calls=3, warmup=1,
+                       label="long-context", state_io_units=H, state_io_count=1)
+    res["workload"] = (f"KDA long-context prefill bf16: B1 H{H} T={T} d128, gate + RMSNorm, zero initial "
+                       f"state, fp32 final state; automatic sequence split")
+    if cpu_ok:
+        import oracle
+        oracle.build()
+        cores = oracle.max_threads()
+        P = min(T, 65536)
+        pre = synth.PrefillInputs(inp.q[:P], inp.k[:P], inp.v[:P], inp.g[:P], inp.beta[:P], inp.gate[:P],
+                                  None, np.array([0, P]))
+        units = [(0, h) for h in range(H)]
+        r, dt, ht = oracle_sample_tokens_per_s(pre, H, units)
+        res["cpu_baseline"] = {"value": r, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": f"the first {P} tokens of all {H} heads ({ht} head-tokens, "
+                                         f"{dt:.1f} s), fp64, OpenMP over the {H} heads"}
+    del inp
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_unbounded(args, L, stream, dev, bounded_ms, rank, w):

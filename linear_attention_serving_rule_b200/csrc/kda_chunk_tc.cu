@@ -939,6 +939,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           at16(sm, OFF_TP + sw128_oct(i, oc, 8192)) = pack8(f);
         }
       }
+      // A partial last chunk: the v tile's rows t >= L hold the next sequence's tokens (or the
+      // zero fill past the tensor).  T' has zero columns there (beta = 0), but 0 * Inf or NaN is
+      // NaN, so the rows are cleared: a sequence must not see its neighbour's values at all.
+      if (need_v && L < C) {
+        if (!wg_wait(&m->full_v, par)) { ok = false; break; }
+        for (int idx = tid; idx < (C - L) * 16; idx += kCompute) {
+          const int t = L + (idx >> 4), c16 = idx & 15;  // a row's 16-byte chunks, either block
+          at16(sm, OFF_V + (c16 >> 3) * 8192 + t * 128 + ((c16 & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
       ops_arrive();  // ---------------------------------------------- UMMA: W = T' Kt, U' = T' V
       if (write_out && j > 0) epilogue_b(L_prev, tok_prev);  // in the shadow of the W|U' UMMAs
       {

@@ -16,6 +16,8 @@
 // warp streams one 512-byte state row per 128-bit load, rows are spread over the 8
 // warps, and the cross-row reductions go through shared memory.  The state is held in
 // registers between the load and the store so it crosses HBM exactly twice.
+#include <atomic>
+
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -213,13 +215,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   }
 }
 
-// CTAs of one kernel instance resident on the whole device at once (cached per device)
+// CTAs of one kernel instance resident on the whole device at once (cached per device; host
+// threads that launch at the same time may each compute it and store the same value)
 template <typename T, int DK, int DV, bool kPre>
 int resident_ctas() {
-  static int cache[64] = {};
+  static std::atomic<int> cache[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (cache[dev] == 0) {
+  int c = cache[dev].load(std::memory_order_relaxed);
+  if (c == 0) {
     int per_sm = 0, sms = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<T, DK, DV, kPre>, kThreads, 0) !=
             cudaSuccess ||
@@ -227,9 +231,10 @@ int resident_ctas() {
       (void)cudaGetLastError();  // no prefetch then; the launch's own error check must not see this
       return 0;
     }
-    cache[dev] = per_sm * sms > 0 ? per_sm * sms : -1;
+    c = per_sm * sms > 0 ? per_sm * sms : -1;
+    cache[dev].store(c, std::memory_order_relaxed);
   }
-  return cache[dev] > 0 ? cache[dev] : 0;
+  return c > 0 ? c : 0;
 }
 
 template <typename T, int DK, int DV, bool kPre>

@@ -72,6 +72,9 @@ struct ChunkParams {
   uint32_t flags;
 };
 
+// Device-side helpers: compiled by nvcc only, so that the host code of the C ABI also builds
+// with a plain C++ compiler (the host-side sanitizer tests do that).
+#ifdef __CUDACC__
 // Set the device error word once (the first error wins).
 __device__ __forceinline__ void report_error(uint32_t* word, kda_status s) {
   if (word) atomicCAS(word, 0u, (uint32_t)s);
@@ -90,6 +93,7 @@ template <>
 __device__ __forceinline__ float from_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+#endif  // __CUDACC__
 
 // Launchers (host).  Each returns cudaSuccess or the launch error.
 cudaError_t launch_decode(const kda_decode_args& a, cudaStream_t stream);

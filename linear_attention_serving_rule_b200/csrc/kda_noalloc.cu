@@ -5,7 +5,12 @@
 // starts.  For them the scratch that kda_chunk_fwd needs lives in a file-scope device array,
 // created with the module on every GPU that loads this library and held until exit.  In host
 // code the array's name is only a host-side handle, so its device address is looked up once per
-// device (with that device current) and handed to kda_chunk_fwd as the workspace.
+// device (with that device current) and handed to kda_chunk_fwd as the workspace.  The address
+// belongs to the device's current context: if that context is destroyed and re-created (a
+// cudaDeviceReset, for instance), the module is loaded again at another address, so the cached
+// address is keyed on the context's unique id as well and looked up again when the id changes.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "kda_internal.cuh"
@@ -17,6 +22,36 @@ static __device__ __align__(256) unsigned char g_kda_scratch[KDA_NOALLOC_SCRATCH
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // id of the context the address belongs to
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if it cannot be read).  The runtime has
+// made the device's primary context current by the time this runs (cudaGetDevice and
+// cudaGetSymbolAddress initialise it).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {  // under g_mu
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+    (void)cudaGetLastError();
+    looked_up = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur && get_id && get_cur(&ctx) == CUDA_SUCCESS && ctx && get_id(ctx, &id) == CUDA_SUCCESS) return id;
+  return 0;
+}
 
 }  // namespace
 
@@ -31,10 +66,13 @@ extern "C" kda_status kda_chunk_fwd_noalloc(const kda_chunk_args* args, void* cu
   void* ptr = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    // (an id of 0, if the driver cannot report one, means: look the address up on every call)
+    const unsigned long long ctx = current_context_id();
+    if (!g_scratch_ptr[dev] || ctx == 0 || ctx != g_scratch_ctx[dev]) {
       void* p = nullptr;
       if (cudaGetSymbolAddress(&p, g_kda_scratch) != cudaSuccess || !p) return KDA_ERR_CUDA;
       g_scratch_ptr[dev] = p;
+      g_scratch_ctx[dev] = current_context_id();
     }
     ptr = g_scratch_ptr[dev];
   }

@@ -104,3 +104,34 @@ def test_prefill_then_decode_equals_longer_prefill(flags):
                                 gate=full.gate[sl])
     assert rel_l2(host(o_dec), host(o_full[sl])) <= TOL_OUT_BF16
     assert rel_l2(host(f_pre), host(f_full)) <= TOL_STATE_BF16
+
+
+def test_decode_1000_steps_sampled_sequences():
+    """The benchmark's decode loop: N512 x H32, 1,000 consecutive in-place steps over a ring of 16
+    input sets, every step on the whole batch.  Four sampled sequences (all heads) are replayed
+    by the oracle step by step; the outputs of the last step and the states after it must agree."""
+    cfg = synth.WORKLOADS["decode_bf16"]
+    N, H, dk, dv, ring = cfg["N"], cfg["H"], cfg["dk"], cfg["dv"], cfg["ring"]
+    steps = cfg["steps"]
+    seed = cfg["seed"]
+    state = synth.make_states(slots=N, H=H, dk=dk, dv=dv, seed=seed, device="cuda")
+    picks = np.array([0, 137, 300, 511])
+    s64 = state[picks].double().cpu().numpy()
+    toks = [synth.make_decode_token(N=N, H=H, dk=dk, dv=dv, seed=seed + 1 + i, device="cuda")
+            for i in range(ring)]
+    sub = [{n: host(getattr(t, n))[picks] for n in ("q", "k", "v", "g", "beta", "gate")} for t in toks]
+    out = torch.empty((N, H, dv), dtype=torch.bfloat16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for i in range(steps):
+        t = toks[i % ring]
+        kda.kda_decode_step(t.q, t.k, t.v, t.g, t.beta, state, gate=t.gate, out=out, error_word=err)
+    torch.cuda.synchronize()
+    assert kda.kda_read_device_error(err) == kda.KDA_OK
+    for i in range(steps):
+        a = sub[i % ring]
+        o_ref = oracle.decode_step(a["q"], a["k"], a["v"], a["g"], a["beta"], s64, gate=a["gate"])
+    assert rel_l2(host(out[picks]), o_ref) <= TOL_OUT_BF16
+    got = state[picks].cpu().numpy()
+    assert rel_l2(got, s64) <= TOL_STATE_BF16
+    for j in range(len(picks)):  # per sequence
+        assert rel_l2(got[j], s64[j]) <= TOL_STATE_BF16, picks[j]

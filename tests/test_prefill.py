@@ -211,3 +211,27 @@ def test_forced_timeout_reports_and_recovers():
     o_ref, f_ref = oracle_full(inp)
     assert rel_l2(host(out), o_ref) <= TOL_OUT_BF16
     assert rel_l2(host(fin), f_ref) <= TOL_STATE_BF16
+
+
+@pytest.mark.parametrize("path", list(PATHS))
+def test_varlen_neighbour_nan_does_not_leak(path):
+    """Packed sequences are independent.  The middle sequence holds NaN in every input; the last,
+    partial chunk of the sequence before it is staged as a full tile that overlaps the NaN rows.
+    Its neighbours' outputs and states must stay finite and match the oracle."""
+    lengths = np.array([100, 77, 150])
+    inp = synth.make_prefill(H=2, dk=128, dv=128, dtype="bf16", seed=38, device="cuda",
+                             lengths=lengths, gate=True, init_state=True)
+    cu = inp.cu_seqlens
+    bad = slice(cu[1], cu[2])
+    for t in (inp.q, inp.k, inp.v, inp.g, inp.gate):
+        t[bad] = float("nan")
+    inp.beta[bad] = float("nan")
+    out, fin = _run(inp, flags=PATHS[path])
+    for n in (0, 2):
+        sl = slice(cu[n], cu[n + 1])
+        one = synth.PrefillInputs(inp.q[sl], inp.k[sl], inp.v[sl], inp.g[sl], inp.beta[sl],
+                                  inp.gate[sl], inp.initial_state[n:n + 1], np.array([0, lengths[n]]))
+        o_ref, f_ref = oracle_full(one)
+        assert torch.isfinite(out[sl]).all() and torch.isfinite(fin[n]).all(), n
+        assert rel_l2(host(out[sl]), o_ref) <= TOL_OUT_BF16, n
+        assert rel_l2(host(fin[n]), f_ref[0]) <= TOL_STATE_BF16, n
