@@ -221,9 +221,9 @@ def oracle_sample_tokens_per_s(inp, H, units, num_threads=0):
 
 
 def cpu_sample_units(B, H, cores):
-    per_core = 2
-    n = max(1, min(B * H, per_core * max(1, cores)))
-    return [(u // H, u % H) for u in range(n)]
+    """The whole batch: the oracle takes about a second for all B x H units on a 16-core host,
+    well inside the bounded CPU sample the benchmark allows."""
+    return [(u // H, u % H) for u in range(B * H)]
 
 
 # ------------------------------------------------------------------ reference arm
@@ -595,7 +595,7 @@ def run_decode(args, dev, stream, rank, world, peaks, peak_src, clocks):
             "gpu_launches": steps}
 
 
-def decode_cpu_baseline(state, toks, N, H, dk, dv, ring, n_seq=64, steps=16):
+def decode_cpu_baseline(state, toks, N, H, dk, dv, ring, n_seq=512, steps=32):
     """The fp64 oracle's decode step on a sample of the batch (n_seq sequences, all heads, `steps`
     consecutive steps over the same input ring), on the host cores: state GB/s in the GPU metric's
     unit (fp32 state bytes read + written per step) and tokens/s."""
@@ -696,7 +696,7 @@ def run_varlen(args, L, stream, dev, rank, world, peaks, peak_src, cpu_ok):
         oracle.build()
         cores = oracle.max_threads()
         rng = np.random.default_rng(5)
-        units = [(int(n), int(h)) for n, h in zip(rng.integers(N, size=2 * cores), rng.integers(H, size=2 * cores))]
+        units = [(int(n), int(h)) for n, h in zip(rng.integers(N, size=512), rng.integers(H, size=512))]
         r, dt, ht = oracle_sample_tokens_per_s(inp, H, units)
         res["cpu_baseline"] = {"value": r, "unit": UNIT, "cores": cores, "kind": "oracle",
                                "sample": f"{len(units)} random (sequence, head) units of this batch "

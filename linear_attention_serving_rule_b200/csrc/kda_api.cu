@@ -74,6 +74,37 @@ kda_status validate(const kda_chunk_args* a) {
 
 int32_t round_up(int64_t x, int32_t m) { return (int32_t)(((x + m - 1) / m) * m); }
 
+// bf16 with dk = dv = 128 runs on the tensor cores; everything else (and the unbounded-decay
+// path) on the fp32 CUDA-core kernel.
+bool uses_tensor_cores(const kda_chunk_args* a) {
+  return a->dtype == KDA_BF16 && a->dk == 128 && a->dv == 128 &&
+         !(a->flags & (KDA_FLAG_FORCE_SIMT | KDA_FLAG_UNBOUNDED_DECAY));
+}
+
+int64_t waves(int64_t units) { return (units + kPlanSMs - 1) / kPlanSMs; }
+
+// Automatic segment count for `busy` (sequence, head) units of one long length: the split runs
+// launch A (each sequence's first segment in full, and pass 1 of the middle segments: two units
+// each on the tensor cores, S_loc and the transition M; one augmented unit on the CUDA cores,
+// launched on its own), the combine, and launch B (the other segments from their start states).
+// Every unit of a launch takes the time of one segment, so the call takes about
+// (waves of A + waves of B) / P of the unsplit time; the P with the least is taken, if it
+// saves at least a fifth.
+int32_t auto_segments(int64_t busy, bool tc) {
+  int32_t best = 1;
+  double best_t = 0.8;
+  for (int32_t P = 2; P <= 64; ++P) {
+    const int64_t w = tc ? waves(busy * (1 + 2 * (int64_t)(P - 2)))
+                         : waves(busy) + (P > 2 ? waves(busy * (int64_t)(P - 2)) : 0);
+    const double t = (double)(w + waves(busy * (int64_t)(P - 1))) / P;
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best = P;
+    }
+  }
+  return best;
+}
+
 Layout make_layout(const kda_chunk_args* a) {
   Layout L;
   const int32_t N = a->num_seqs;
@@ -95,7 +126,7 @@ Layout make_layout(const kda_chunk_args* a) {
   int32_t P = 1;
   bool auto_mode = a->split_segments == 0;
   if (auto_mode) {
-    if (busy > 0 && busy * 2 <= kPlanSMs) P = (int32_t)std::min<int64_t>(64, kPlanSMs / busy);
+    if (busy > 0 && busy * 2 <= kPlanSMs) P = auto_segments(busy, uses_tensor_cores(a));
   } else {
     P = a->split_segments;
   }
@@ -239,14 +270,15 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
   if (cudaMemsetAsync(a->workspace, 0, sizeof(uint32_t), stream) != cudaSuccess) return KDA_ERR_CUDA;
   if (a->num_seqs == 0) return KDA_OK;
 
-  // bf16 with dk = dv = 128 runs on the tensor cores; everything else (and the split's
-  // augmented pass 1) on the fp32 CUDA-core kernel.
-  const bool use_tc = a->dtype == KDA_BF16 && a->dk == 128 && a->dv == 128 &&
-                      !(a->flags & (KDA_FLAG_FORCE_SIMT | KDA_FLAG_UNBOUNDED_DECAY));
+  const bool use_tc = uses_tensor_cores(a);
 
-  // Pass 1 of split sequences: the head segment from the true initial state, and the
-  // other non-final segments from [0 | I] (local state and transition matrix).
-  std::vector<Seg> head, local, whole;
+  // Launch A: every unsplit sequence, and the first segment of each split sequence, in full from
+  // its initial state (outputs, snapshots; a first segment also leaves its end state in the
+  // workspace as the second segment's start state); with them pass 1 of the middle segments
+  // (local state from zero and the transition matrix; on the CUDA cores as one augmented unit,
+  // launched on its own because its kernel differs).  Then the combine, then launch B: the
+  // remaining segments of the split sequences from their start states.
+  std::vector<Seg> first, local, rest;
   std::vector<int64_t> snap_base;
   if (a->snapshots) snap_base = snapshot_bases(L, a->snapshot_interval, nullptr);
   // segments that carry the true state write the snapshots inside them
@@ -258,30 +290,29 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
     const SeqSpan& sp = L.seqs[n];
     const int32_t np = L.nseg[n];
     if (np == 1) {
-      whole.push_back(with_snap(make_seg(sp.tok0, sp.len, sp.seq, kRoleWhole, -1, 1), n));
+      first.push_back(with_snap(make_seg(sp.tok0, sp.len, sp.seq, kRoleWhole, -1, 1), n));
       continue;
     }
     const int32_t sl = L.seglen[n], b = L.slot0[n];
     for (int32_t q = 0; q < np; ++q) {
       const int32_t t0 = sp.tok0 + q * sl;
       const int32_t len = std::min(sl, sp.len - q * sl);
-      if (q == 0) {
-        head.push_back(make_seg(t0, len, sp.seq, kRoleHead, b, 0));
-      } else if (q < np - 1) {
+      if (q == 0) {  // in full; its end state -> start-state slot b + 1
+        first.push_back(with_snap(make_seg(t0, len, sp.seq, kRoleWhole, b, 0), n));
+        continue;
+      }
+      if (q < np - 1) {
         if (use_tc) {  // S_loc and M as two plain-state units of the tensor-core kernel
-          local.push_back(make_seg(t0, len, sp.seq, kRoleLocalS, b + q, 0));
-          local.push_back(make_seg(t0, len, sp.seq, kRoleLocalM, b + q, 0));
+          first.push_back(make_seg(t0, len, sp.seq, kRoleLocalS, b + q, 0));
+          first.push_back(make_seg(t0, len, sp.seq, kRoleLocalM, b + q, 0));
         } else {
           local.push_back(make_seg(t0, len, sp.seq, kRoleLocal, b + q, 0));
         }
       }
-      // the first segment's snapshots come from its pass-2 run (kRoleWhole from the initial state)
-      if (q == 0) whole.push_back(with_snap(make_seg(t0, len, sp.seq, kRoleWhole, b, 0), n));
-      else whole.push_back(with_snap(make_seg(t0, len, sp.seq, kRoleFromWs, b + q, q == np - 1 ? 1 : 0), n));
+      rest.push_back(with_snap(make_seg(t0, len, sp.seq, kRoleFromWs, b + q, q == np - 1 ? 1 : 0), n));
     }
   }
-  cudaError_t e = cudaSuccess;
-  if (!head.empty()) e = run_segments(head, p, a->dtype, use_tc, stream);
+  cudaError_t e = run_segments(first, p, a->dtype, use_tc, stream);
   if (e == cudaSuccess && !local.empty()) e = run_segments(local, p, a->dtype, use_tc, stream);
   if (e == cudaSuccess && L.any_split) {
     // combine: S_start(q+1) = M_q S_start(q) + S_loc(q), sequential over q per (sequence, head)
@@ -298,7 +329,7 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
     }
     if (e == cudaSuccess && plan.n_seg > 0) e = launch_split_combine(plan, p, 0, stream);
   }
-  if (e == cudaSuccess) e = run_segments(whole, p, a->dtype, use_tc, stream);
+  if (e == cudaSuccess && !rest.empty()) e = run_segments(rest, p, a->dtype, use_tc, stream);
   return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

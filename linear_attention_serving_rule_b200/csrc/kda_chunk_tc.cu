@@ -74,7 +74,7 @@ constexpr uint32_t OFF_S = 155648;   // bf16 state, MN-major [dk rows][dv], two 
 constexpr uint32_t OFF_TP = 188416;  // T' = T Diag(beta), bf16 [64][64]
 constexpr uint32_t OFF_P = 196608;   // P (causally masked), bf16 [64][64]
 constexpr uint32_t OFF_MISC = 204800;
-constexpr uint32_t OFF_GATE = OFF_MISC + 8192;  // gate logits of the chunk whose epilogue is pending
+constexpr uint32_t OFF_GATE = OFF_MISC + 8192;  // gate logits of the chunk whose epilogue is pending (TMA)
 constexpr uint32_t SMEM_BYTES = OFF_GATE + 16384 + 1024;
 static_assert(SMEM_BYTES <= 232448, "over the 227 KB of shared memory a block may use");
 // fp32 L = Diag(beta) A [64][68], then fp32 T [64][68]: a row stride of 4 mod 32 words keeps the
@@ -95,6 +95,7 @@ struct Misc {
   // k and q have their own barriers: the k rows are free after the W|U' UMMAs, the q rows only
   // after the U/O UMMAs
   uint64_t full_g, full_k, full_q, full_v, empty_g, empty_k, empty_q, empty_v, mma, ops;
+  uint64_t full_gate, empty_gate;  // the gate tile: loaded per chunk, freed after its epilogue
   uint32_t tmem_base;
   int32_t abort;
   float beta[2][C];  // double-buffered by chunk parity (written by the producer warp)
@@ -109,7 +110,7 @@ static_assert(offsetof(Misc, nw) % 16 == 0, "float4 reads of the norm weight nee
 static_assert(offsetof(Misc, full_g) % 8 == 0, "mbarriers need 8-byte alignment");
 
 struct TcMaps {
-  CUtensorMap q, k, g, v;
+  CUtensorMap q, k, g, v, gate;  // gate: only when the call has gate logits
 };
 static_assert(sizeof(Plan) + sizeof(TcMaps) + sizeof(ChunkParams) + 128 <= 32764,
               "kernel parameters exceed the 32,764-byte limit");
@@ -169,6 +170,11 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 __device__ __forceinline__ uint4& at16(uint8_t* base, uint32_t off) { return *reinterpret_cast<uint4*>(base + off); }
@@ -257,11 +263,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t drain_limit = 2000000000ull;
   const int nchunks = (seg.len + C - 1) / C;
   const bool need_v = seg.role != kRoleLocalM;  // the transition pass runs with values = 0
+  const bool write_out = (seg.role == kRoleWhole || seg.role == kRoleFromWs);
+  const bool stage_gate = write_out && has_gate;  // the epilogue needs the chunk's gate logits
 
   if (tid == 0) {
     mbar_init(&m->full_g, 1); mbar_init(&m->full_k, 1); mbar_init(&m->full_q, 1); mbar_init(&m->full_v, 1);
     mbar_init(&m->empty_g, 1); mbar_init(&m->empty_k, 1); mbar_init(&m->empty_q, 1); mbar_init(&m->empty_v, 1);
     mbar_init(&m->mma, 1);
+    mbar_init(&m->full_gate, 1);
+    mbar_init(&m->empty_gate, 1);
     mbar_init(&m->ops, 8);  // one arrival per compute warp: a UMMA group's operands are in place
     m->abort = 0;
     fence_mbar_init();
@@ -272,6 +282,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 8 && lane == 0) {
     prefetch_tmap(&maps.q); prefetch_tmap(&maps.k); prefetch_tmap(&maps.g); prefetch_tmap(&maps.v);
+    if (stage_gate) prefetch_tmap(&maps.gate);
   }
   if (tid < DV) m->nw[tid] = p.norm_weight ? p.norm_weight[tid] : 1.f;
   tc_fence_before();
@@ -283,7 +294,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ===================================================================== TMA producer
     // Lane 0 issues the tile loads; the whole warp first fetches the chunk's beta into the
     // double buffer m->beta[j & 1], published by the same mbarrier as the g tile.
-    int ig = -1, ik = -1, iq = -1, iv = -1;  // last chunk whose g, k, q and v loads were issued
+    int ig = -1, ik = -1, iq = -1, iv = -1, igt = -1;  // last chunk whose g, k, q, v, gate loads were issued
+    auto load_gate = [&](int jg) -> bool {  // lane 0
+      if (!wait_bounded(&m->empty_gate, (uint32_t)((jg & 1) ^ 1), m, drain_limit, p.error_word)) return false;
+      mbar_arrive_expect_tx(&m->full_gate, 16384);
+      for (int hf = 0; hf < 2; ++hf)
+        tma_load_3d(sm + OFF_GATE + hf * 8192, &maps.gate, &m->full_gate, hf * 64, h, seg.tok0 + jg * C);
+      igt = jg;
+      return true;
+    };
+    bool prod_ok = true;
     for (int j = 0; j < nchunks; ++j) {
       const int32_t tok = seg.tok0 + j * C;
       const int L = min(C, seg.len - j * C);
@@ -314,6 +334,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hf = 0; hf < 2; ++hf) tma_load_3d(sm + OFF_G + hf * 8192, &maps.g, &m->full_g, hf * 64, h, tok);
       }
       ig = j;
+      // the previous chunk's gate logits (its epilogue runs beside this chunk's Gram and W|U'
+      // UMMAs): the buffer frees once the epilogue of the chunk before it is done, which is when
+      // this chunk's k rows free too, so waiting for it here delays nothing
+      if (stage_gate && j > 0) {
+        if (lane == 0) okw = load_gate(j - 1) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        if (!okw) break;
+      }
       if (lane == 0) okw = wait_bounded(&m->empty_k, par, m, drain_limit, p.error_word) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);
       if (!okw) break;
@@ -341,8 +369,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       iv = j;
     }
+    prod_ok = *(volatile int32_t*)&m->abort == 0;
+    // the last chunk's gate logits
+    if (stage_gate && nchunks > 0 && prod_ok && lane == 0) load_gate(nchunks - 1);
+    __syncwarp();
     // drain: after an abort, wait (bounded, regardless of the abort) for the loads issued
     if (lane == 0 && *(volatile int32_t*)&m->abort) {
+      if (igt >= 0) wait_bounded(&m->full_gate, (uint32_t)(igt & 1), m, drain_limit, p.error_word, false);
       if (ig >= 0) wait_bounded(&m->full_g, (uint32_t)(ig & 1), m, drain_limit, p.error_word, false);
       if (ik >= 0) wait_bounded(&m->full_k, (uint32_t)(ik & 1), m, drain_limit, p.error_word, false);
       if (iq >= 0) wait_bounded(&m->full_q, (uint32_t)(iq & 1), m, drain_limit, p.error_word, false);
@@ -359,17 +392,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t hi = 16u << 16;
       for (int j = 0; j < nchunks; ++j) {
         const uint32_t par = (uint32_t)(j & 1);
-        // A | P over the stacked Kc operand, as two N=80 halves (Kc rows 0-79 and 80-159; row 80
-        // starts a swizzle atom) whose K steps interleave
+        // A | P over the stacked Kc operand: one N=160 chain.  The issuing thread waits about the
+        // same time per K step whatever N is, so one wide chain beats two interleaved N=80 halves
+        // (measured 1.6 K against 2.4 K cycles for the group alone).
         if (!wait_bounded(&m->ops, (oph++) & 1u, m, limit, p.error_word)) break;
         tc_fence_after();
         {
-          const uint32_t id = idesc_bf16_f32(128, KC_ROWS / 2, 0, 0);
-          const UChain c[2] = {
-              uchain(tmem + TM_AP, sm_u + OFF_KL, 16, true, 16384, sm_u + OFF_KC, 16, true, KC_BLK, id, false),
-              uchain(tmem + TM_AP + KC_ROWS / 2, sm_u + OFF_KL, 16, true, 16384, sm_u + OFF_KC + (KC_ROWS / 2) * 128, 16,
-                     true, KC_BLK, id, false)};
-          umma_interleaved(c, 8);
+          const uint64_t a0 = smem_desc_sw128(sm_u + OFF_KL, 16, 1024), b0 = smem_desc_sw128(sm_u + OFF_KC, 16, 1024);
+          const uint32_t id = idesc_bf16_f32(128, KC_ROWS, 0, 0);
+#pragma unroll 1
+          for (int k = 0; k < 8; ++k)  // (a rolled loop: each step waits ~180 cycles anyway)
+            umma_bf16(tmem + TM_AP, a0 + (((k >> 2) * 16384u + (k & 3) * 32u) >> 4),
+                      b0 + (((k >> 2) * KC_BLK + (k & 3) * 32u) >> 4), id, k > 0 ? 1u : 0u);
         }
         umma_commit(&m->mma);
         ++committed;
@@ -439,7 +473,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = 32 * q4 + lane;
     const uint32_t tl = tmem + ((uint32_t)(32 * q4) << 16);
     const size_t unit_state = (size_t)DK * DV;
-    const bool write_out = (seg.role == kRoleWhole || seg.role == kRoleFromWs);
     // chunk-boundary snapshot of the state after segment-local token e, or null
     auto snap_dst = [&](int e) -> float* {
       if (seg.snap < 0 || e < seg.snap_off || (e - seg.snap_off) % p.snap_interval != 0) return nullptr;
@@ -467,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- start state -> TMEM + bf16 copy
     {
       const float* src = nullptr;
-      if (seg.role == kRoleWhole || seg.role == kRoleHead) {
+      if (seg.role == kRoleWhole) {
         if (p.initial_state) src = p.initial_state + ((size_t)seg.seq * H + h) * unit_state;
       } else if (seg.role == kRoleFromWs) {
         src = p.ws_state + ((size_t)seg.slot * H + h) * unit_state;
@@ -500,20 +533,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
     }
 
-    // The gate logits of a chunk are staged with cp.async at the start of the next chunk, into
-    // their own buffer: row t at OFF_GATE + 256 t, 16-byte chunk c at position c ^ (t & 15).
-    auto load_gate = [&](int L_e, int32_t tok_e) {
-      if (!has_gate) return;
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int idx = tid + kCompute * r;
-        const int t = idx >> 4, c16 = idx & 15;
-        if (t < L_e)
-          cp_async_16(sm_u + OFF_GATE + t * 256 + ((c16 ^ (t & 15)) << 4),
-                      static_cast<const __nv_bfloat16*>(p.gate) + ((size_t)(tok_e + t) * H + h) * DV + 8 * c16);
-      }
-      cp_async_commit();
-    };
+    // The gate logits of a chunk arrive by TMA (128-byte swizzled [64 tokens][128 B] blocks, one
+    // per 64 columns) while the next chunk's prep runs; epilogue part A waits for them and the
+    // buffer is handed back after part B.
     // Epilogue of one chunk, run by both warpgroups in two parts while the next chunk's UMMAs run:
     // O stays in TMEM columns [416,480) until the next chunk's O UMMAs.  Lanes l < 16 of warp
     // (q, wg) hold columns 32 wg .. 32 wg + 31 and lanes l + 16 columns 64 + 32 wg .. of O row
@@ -534,12 +556,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (has_gate) {
           float gl8[8];
           const int c16 = (c0 >> 3) + oc0 + oc;
-          unpack8(at16(sm, OFF_GATE + t * 256 + ((c16 ^ (t & 15)) << 4)), gl8);
+          unpack8(at16(sm, OFF_GATE + sw128_oct(t, c16, 8192)), gl8);
           const float4 w0 = *reinterpret_cast<const float4*>(&m->nw[c0 + 8 * (oc0 + oc)]);
           const float4 w1 = *reinterpret_cast<const float4*>(&m->nw[c0 + 8 * (oc0 + oc) + 4]);
           const float w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+          // sigmoid(x) = (1 + tanh(x / 2)) / 2: one MUFU operation per element
 #pragma unroll
-          for (int e = 0; e < 8; ++e) f[e] *= __fdividef(w[e], 1.f + ex2(-gl8[e] * kLog2e));
+          for (int e = 0; e < 8; ++e) {
+            const float hw = 0.5f * w[e] * f[e];
+            f[e] = fmaf(hw, tanh_approx(0.5f * gl8[e]), hw);
+          }
         }
         op[oc0 + oc] = pack8(f);
       }
@@ -778,9 +804,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ops_arrive();  // ---------------------------------------------- UMMA: A | P (issued by warp 9)
       // ---------------------------------------------------------------- in the shadow of the Gram UMMAs:
       // the previous chunk's epilogue (its O is still in TMEM)
-      cp_async_wait_all();
-      sync_wg();  // the staged gate logits are visible to every thread
-      if (write_out && j > 0) epilogue_a(L_prev, tok_prev);
+      if (write_out && j > 0) {
+        if (stage_gate && !wg_wait(&m->full_gate, (uint32_t)((j - 1) & 1))) { ok = false; break; }
+        epilogue_a(L_prev, tok_prev);
+      }
       {
         const bool r = wg_wait(&m->mma, mph & 1u);
         ++mph;
@@ -960,6 +987,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid == 0) {  // v and the k rows (e^{gamma} k in place) consumed
         if (need_v) mbar_arrive(&m->empty_v);
         mbar_arrive(&m->empty_k);
+        if (stage_gate && j > 0) mbar_arrive(&m->empty_gate);  // chunk j - 1's epilogue is done
       }
 
       // ---------------------------------------------------------------- -W -> bf16
@@ -1028,9 +1056,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       ops_arrive();  // ---------------------------------------------- UMMA: O += P U ; S += Kh^T U
-      // in their shadow: stage this chunk's gate logits for its epilogue (the buffer's previous
-      // contents were consumed beside this chunk's W|U' UMMAs)
-      if (write_out) load_gate(L, tok);
       {
         const bool r = wg_wait(&m->mma, mph & 1u);
         ++mph;
@@ -1042,19 +1067,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       tok_prev = tok;
     }
     if (ok && write_out && nchunks > 0) {
-      cp_async_wait_all();
-      sync_wg();
-      epilogue_a(L_prev, tok_prev);
-      epilogue_b(L_prev, tok_prev);
+      ok = !stage_gate || wg_wait(&m->full_gate, (uint32_t)((nchunks - 1) & 1));
+      if (ok) {
+        epilogue_a(L_prev, tok_prev);
+        epilogue_b(L_prev, tok_prev);
+      }
     }
 
     // ---------------------------------------------------------------- end state
     if (ok) {
       float* dst = nullptr;
       if (seg.role == kRoleWhole || seg.role == kRoleFromWs) {
-        if (seg.last && p.final_state) dst = p.final_state + ((size_t)seg.seq * H + h) * unit_state;
-      } else if (seg.role == kRoleHead) {
-        dst = p.ws_state + ((size_t)(seg.slot + 1) * H + h) * unit_state;
+        if (seg.last) {
+          if (p.final_state) dst = p.final_state + ((size_t)seg.seq * H + h) * unit_state;
+        } else if (seg.role == kRoleWhole) {  // first segment of a split sequence: the next one's start
+          dst = p.ws_state + ((size_t)(seg.slot + 1) * H + h) * unit_state;
+        }
       }
       size_t ld = DV;
       if (seg.role == kRoleLocalS || seg.role == kRoleLocalM) {  // (S_loc | M) block, row stride dv + dk
@@ -1079,7 +1107,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    cp_async_wait_all();  // no gate copy may outlive the block (after an abort)
   }
   tc_fence_before();
   __syncthreads();
@@ -1127,7 +1154,7 @@ cudaError_t launch_chunk_tc(const Plan& plan, const ChunkParams& p, cudaStream_t
   memset(&maps, 0, sizeof(maps));
   const int64_t T = p.total_tokens;
   if (!make_map(&maps.q, p.q, p.H, T) || !make_map(&maps.k, p.k, p.H, T) || !make_map(&maps.g, p.g, p.H, T) ||
-      !make_map(&maps.v, p.v, p.H, T))
+      !make_map(&maps.v, p.v, p.H, T) || (p.gate && !make_map(&maps.gate, p.gate, p.H, T)))
     return cudaErrorInvalidValue;
   const bool pre = (p.flags & (KDA_FLAG_G_LOGITS | KDA_FLAG_QK_L2NORM)) != 0;
   auto kern = pre ? chunk_tc_kernel<true> : chunk_tc_kernel<false>;

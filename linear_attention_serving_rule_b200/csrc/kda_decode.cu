@@ -19,9 +19,12 @@
 #include <atomic>
 
 #include "kda_internal.cuh"
+#include "ptx_sm100.cuh"
 
 namespace kda {
 namespace {
+
+using namespace ptx;
 
 constexpr int kThreads = 256;
 
@@ -43,6 +46,16 @@ struct DecodeParams {
   uint32_t flags;
   uint32_t* error_word;
 };
+
+// Two fp32 fused multiply-adds at once (fma.rn.f32x2: each half rounds like fma.rn.f32).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(*reinterpret_cast<const uint64_t*>(&a)),
+      "l"(*reinterpret_cast<const uint64_t*>(&b)), "l"(*reinterpret_cast<const uint64_t*>(&c)));
+  return *reinterpret_cast<const float2*>(&r);
+}
+__device__ __forceinline__ float2 lo2(const float4& v) { return make_float2(v.x, v.y); }
+__device__ __forceinline__ float2 hi2(const float4& v) { return make_float2(v.z, v.w); }
 
 // Bulk prefetch of [addr, addr + bytes) into L2 (a hint: no completion, no shared memory).
 __device__ __forceinline__ void prefetch_l2(const void* addr, uint32_t bytes) {
@@ -215,6 +228,344 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
   }
 }
 
+// K > 1 tokens per sequence (speculative verification): the state is read once and written once,
+// and the K tokens need only a few block-wide barriers per group of up to KG tokens instead of three
+// per token.  With S0 the state before the group, G_j the per-channel cumulative log-decay from the
+// group start through token j, and k, q as the recurrence uses them (L2-normalised with
+// KDA_FLAG_QK_L2NORM), unrolling the recurrence gives, for j = 1 .. Kg,
+//
+//   S'_j^T k_j = S0^T (e^{G_j} k_j) + sum_{i<j} u_i c_ji,   c_ji = sum_c k_i[c] k_j[c] e^{G_j[c] - G_i[c]}
+//   u_j        = beta_j (v_j - S'_j^T k_j)
+//   o_j        = scale (S0^T (e^{G_j} q_j) + sum_{i<=j} u_i d_ji),   d_ji likewise with q_j (d_jj = k_j . q_j)
+//   S_j        = Diag(e^{g_j}) S_{j-1} + k_j u_j^T
+//
+// (S'_j = Diag(e^{g_j}) S_{j-1} is the state the delta rule reads before token j's write).  So one
+// pass over the registers forms all 2 Kg column reductions S0^T (e^{G_j} k_j), S0^T (e^{G_j} q_j),
+// the small Kg x Kg dots c, d come from the token vectors alone, the u_j and o_j follow column by
+// column without further barriers, and the state is then updated token by token in registers (no
+// reductions), writing each position's state when asked.  Every input of a group is fetched with
+// cp.async before anything waits on it (for the first group, before the state is loaded), so a CTA
+// waits for global memory once per group, not once per input.
+constexpr int kMultiGroup = 4;  // tokens per group
+
+template <typename T, int DK, int DV>
+struct MultiSmem {
+  static constexpr int KG = kMultiGroup;
+  static constexpr int RPP = kThreads / (DV / 4);
+  alignas(16) T rk[KG][DK];  // the group's raw token inputs (cp.async)
+  alignas(16) T rq[KG][DK];
+  alignas(16) T rg[KG][DK];
+  alignas(16) T rv[KG][DV];
+  alignas(16) T rgate[KG][DV];
+  float sk[KG][DK], sq[KG][DK];   // k, q as loaded (fp32)
+  float sg[KG][DK], sa[KG][DK];   // cumulative log-decay G_j from the group start; e^{g_j}
+  float skg[KG][DK], sqg[KG][DK]; // k_j e^{G_j}, q_j e^{G_j}
+  float ski[KG][DK];              // k_j e^{-G_j} (bounded decay: |G_j| <= 5 KG, so it stays finite)
+  float wk[KG][DK];               // e^{G_last - G_j} k_j (normalised): the end state's write factors
+  float wK[DK];                   // e^{G_last}: the end state's decay of S0
+  alignas(16) float red[RPP][2 * KG][DV];  // column partial sums; then red[0][2 j] = o_j (see below)
+  alignas(16) float su[KG][DV];
+  float sdot[KG][KG][2];          // [j][i]: raw c_ji (i < j), raw d_ji (i <= j)
+  float snrm[KG][2];              // |k_j|^2, |q_j|^2
+  float sbeta[KG];
+};
+
+template <typename T, int DK, int DV, bool kPre>
+__global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const DecodeParams p) {
+  constexpr int KG = kMultiGroup;
+  constexpr int TPR = DV / 4;              // threads per state row (one float4 each)
+  constexpr int RPP = kThreads / TPR;      // rows per pass
+  constexpr int NP = DK / RPP;             // passes (float4 registers per thread)
+  static_assert(DK % RPP == 0, "rows must divide evenly");
+  extern __shared__ __align__(16) uint8_t dsm[];
+  MultiSmem<T, DK, DV>& sm = *reinterpret_cast<MultiSmem<T, DK, DV>*>(dsm);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int unit = blockIdx.x;
+  const int n = unit / p.H;
+  const int h = unit - n * p.H;
+  const bool checked = (p.flags & KDA_FLAG_CHECK_DECAY) != 0;
+  const bool g_logits = kPre && (p.flags & KDA_FLAG_G_LOGITS) != 0;
+  const bool l2norm = kPre && (p.flags & KDA_FLAG_QK_L2NORM) != 0;
+  const bool b_logits = kPre && (p.flags & KDA_FLAG_BETA_LOGITS) != 0;
+  const int K = p.tokens;
+
+  int slot = p.state_indices ? p.state_indices[n] : n;
+  if (slot < 0 || slot >= p.num_slots) {  // uniform over the block
+    if (tid == 0) report_error(p.error_word, KDA_ERR_BAD_STATE_INDEX);
+    return;
+  }
+  // the token inputs of the group starting at `base`: 16-byte cp.async chunks, then beta
+  constexpr int CK = DK * (int)sizeof(T) / 16, CV = DV * (int)sizeof(T) / 16;  // chunks per row
+  float beta_reg = 0.f;
+  auto fetch_group = [&](int base) {
+    const int Kg = min(KG, K - base);
+    for (int idx = tid; idx < Kg * (3 * CK + 2 * CV); idx += kThreads) {
+      const int j = idx / (3 * CK + 2 * CV);
+      int c = idx - j * (3 * CK + 2 * CV);
+      const size_t row = ((size_t)n * K + base + j) * p.H + h;  // token inputs are [N, K, H, d]
+      const T* src;
+      uint8_t* dst;
+      if (c < 3 * CK) {
+        const int t = c / CK;
+        c -= t * CK;
+        src = static_cast<const T*>(t == 0 ? p.k : t == 1 ? p.q : p.g) + row * DK;
+        dst = reinterpret_cast<uint8_t*>(t == 0 ? sm.rk[j] : t == 1 ? sm.rq[j] : sm.rg[j]);
+      } else {
+        c -= 3 * CK;
+        const int t = c / CV;
+        c -= t * CV;
+        if (t == 1 && p.gate == nullptr) continue;
+        src = static_cast<const T*>(t == 0 ? p.v : p.gate) + row * DV;
+        dst = reinterpret_cast<uint8_t*>(t == 0 ? sm.rv[j] : sm.rgate[j]);
+      }
+      cp_async_16(smem_u32(dst + 16 * c), reinterpret_cast<const uint8_t*>(src) + 16 * c);
+    }
+    cp_async_commit();
+    if (tid < Kg) beta_reg = to_f32(static_cast<const T*>(p.beta)[((size_t)n * K + base + tid) * p.H + h]);
+  };
+  fetch_group(0);
+
+  float* S = p.state + ((size_t)slot * p.H + h) * (size_t)(DK * DV);
+  const int cg = tid % TPR;   // column group: columns 4cg .. 4cg+3
+  const int r0 = tid / TPR;   // first row; rows r0 + RPP * i
+  float4 s[NP];
+#pragma unroll
+  for (int i = 0; i < NP; ++i)
+    s[i] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)(r0 + RPP * i) * DV) + cg);
+  if (tid == 0 && p.ahead > 0 && unit + p.ahead < (int)gridDim.x) {  // see decode_kernel
+    const int u2 = unit + p.ahead;
+    const int n2 = u2 / p.H;
+    const int slot2 = p.state_indices ? p.state_indices[n2] : n2;
+    if (slot2 >= 0 && slot2 < p.num_slots)
+      prefetch_l2(p.state + ((size_t)slot2 * p.H + (u2 - n2 * p.H)) * (size_t)(DK * DV),
+                  (uint32_t)(DK * DV * sizeof(float)));
+  }
+
+  const bool commit = (p.flags & KDA_FLAG_DECODE_NO_COMMIT) == 0;
+  for (int base = 0; base < K; base += KG) {
+    const int Kg = min(KG, K - base);
+    if (base > 0) {
+      __syncthreads();  // the previous group's shared arrays are consumed
+      fetch_group(base);
+    }
+    cp_async_wait_all();
+    if (tid < Kg) sm.sbeta[tid] = b_logits ? 1.f / (1.f + __expf(-beta_reg)) : beta_reg;  // beta = sigmoid(b)
+    __syncthreads();
+    // ---- per channel: G_j (prefix over the group), e^{g_j}, and the decayed k, q
+    if (tid < DK) {
+      float acc = 0.f;
+      for (int j = 0; j < Kg; ++j) {
+        const float kx = to_f32(sm.rk[j][tid]), qx = to_f32(sm.rq[j][tid]);
+        float gi = to_f32(sm.rg[j][tid]);
+        if (g_logits) gi = KDA_G_MIN / (1.f + __expf(-gi));  // g = g_min sigmoid(a)
+        if (checked && !(((p.flags & KDA_FLAG_UNBOUNDED_DECAY) || gi >= KDA_G_MIN) && gi <= 0.0f))
+          report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
+        sm.sk[j][tid] = kx;
+        sm.sq[j][tid] = qx;
+        sm.sa[j][tid] = __expf(gi);
+        acc += gi;
+        sm.sg[j][tid] = acc;
+        const float e = __expf(acc);
+        sm.skg[j][tid] = kx * e;
+        sm.sqg[j][tid] = qx * e;
+        sm.ski[j][tid] = kx * __expf(-acc);
+      }
+    }
+    __syncthreads();
+    // ---- the token dots and the column reductions over the state.  The 24 dots of a full group
+    // (d_ji for i <= j, c_ji for i < j, |k_j|^2, |q_j|^2) are shared out three per warp; each is
+    // coded in 6 bits (j, i, kind) and dots of tokens past the group's end are skipped.  With the
+    // bounded decay e^{G_j - G_i} = e^{G_j} e^{-G_i} (both finite); with KDA_FLAG_UNBOUNDED_DECAY
+    // the factor is formed from the difference, which cannot overflow.
+    {
+      const bool unbounded = (p.flags & KDA_FLAG_UNBOUNDED_DECAY) != 0;
+      // kind 0: c_ji (k_i, k_j), 1: d_ji (k_i, q_j), 2: |k_j|^2, 3: |q_j|^2; code = 16 kind + 4 j + i
+      constexpr uint64_t kSlot[3] = {
+          // warp w takes 6-bit code w of each word
+          (uint64_t)0x10 | (uint64_t)0x15 << 6 | (uint64_t)0x1A << 12 | (uint64_t)0x1F << 18 |
+              (uint64_t)0x14 << 24 | (uint64_t)0x18 << 30 | (uint64_t)0x19 << 36 | (uint64_t)0x1C << 42,
+          (uint64_t)0x1D << 0 | (uint64_t)0x1E << 6 | (uint64_t)0x04 << 12 | (uint64_t)0x08 << 18 |
+              (uint64_t)0x09 << 24 | (uint64_t)0x0C << 30 | (uint64_t)0x0D << 36 | (uint64_t)0x0E << 42,
+          (uint64_t)0x20 << 0 | (uint64_t)0x24 << 6 | (uint64_t)0x28 << 12 | (uint64_t)0x2C << 18 |
+              (uint64_t)0x30 << 24 | (uint64_t)0x34 << 30 | (uint64_t)0x38 << 36 | (uint64_t)0x3C << 42};
+#pragma unroll
+      for (int sl = 0; sl < 3; ++sl) {
+        const int code = (int)(kSlot[sl] >> (6 * warp)) & 63;
+        const int kind = code >> 4, j = (code >> 2) & 3, i = code & 3;
+        if (j >= Kg) continue;  // uniform over the warp
+        float acc = 0.f;
+        if (kind >= 2) {
+          const float* x = kind == 3 ? sm.sq[j] : sm.sk[j];
+#pragma unroll
+          for (int c0 = 0; c0 < DK; c0 += 32) acc += x[c0 + lane] * x[c0 + lane];
+        } else {
+          const float* xj = kind == 0 ? sm.skg[j] : sm.sqg[j];
+          if (!unbounded) {
+#pragma unroll
+            for (int c0 = 0; c0 < DK; c0 += 32) acc += sm.ski[i][c0 + lane] * xj[c0 + lane];
+          } else {
+            const float* yj = kind == 0 ? sm.sk[j] : sm.sq[j];
+#pragma unroll
+            for (int c0 = 0; c0 < DK; c0 += 32) {
+              const int c = c0 + lane;
+              acc += sm.sk[i][c] * yj[c] * __expf(sm.sg[j][c] - sm.sg[i][c]);
+            }
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) {
+          if (kind < 2) sm.sdot[j][i][kind] = acc;
+          else sm.snrm[j][kind - 2] = acc;
+        }
+      }
+    }
+    // (two tokens per pass over the registers, to keep the accumulators few; column pairs through
+    // the two-wide fp32 FMA)
+#pragma unroll
+    for (int jp = 0; jp < KG; jp += 2) {
+      if (jp >= Kg) break;
+      float2 acc[4][2];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) acc[m][0] = acc[m][1] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < NP; ++i) {
+        const int r = r0 + RPP * i;
+        const float2 sl = lo2(s[i]), sh = hi2(s[i]);
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int j = jp + jj;
+          if (j < Kg) {
+            const float kr = sm.skg[j][r], qr = sm.sqg[j][r];
+            const float2 k2 = make_float2(kr, kr), q2 = make_float2(qr, qr);
+            acc[2 * jj][0] = ffma2(sl, k2, acc[2 * jj][0]);
+            acc[2 * jj][1] = ffma2(sh, k2, acc[2 * jj][1]);
+            acc[2 * jj + 1][0] = ffma2(sl, q2, acc[2 * jj + 1][0]);
+            acc[2 * jj + 1][1] = ffma2(sh, q2, acc[2 * jj + 1][1]);
+          }
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m)
+        if (2 * jp + m < 2 * Kg)
+          reinterpret_cast<float4*>(sm.red[r0][2 * jp + m])[cg] =
+              make_float4(acc[m][0].x, acc[m][0].y, acc[m][1].x, acc[m][1].y);
+    }
+    __syncthreads();
+    // ---- column by column: u_j and o_j for the group's tokens in order (o_j goes to red[0][2 j],
+    // whose column tid only this thread reads, before it writes it)
+    if (tid < DV) {
+      float u[KG];
+#pragma unroll
+      for (int j = 0; j < KG; ++j) {
+        if (j >= Kg) break;
+        float a = 0.f, bq = 0.f;
+#pragma unroll
+        for (int r = 0; r < RPP; ++r) { a += sm.red[r][2 * j][tid]; bq += sm.red[r][2 * j + 1][tid]; }
+        const float rkj = l2norm ? rsqrtf(sm.snrm[j][0] + KDA_L2NORM_EPS) : 1.f;
+        const float rqj = l2norm ? rsqrtf(sm.snrm[j][1] + KDA_L2NORM_EPS) : 1.f;
+        float pred = a * rkj, o = bq * rqj;
+#pragma unroll
+        for (int i = 0; i < KG; ++i) {
+          if (i >= j) break;
+          const float rki = l2norm ? rsqrtf(sm.snrm[i][0] + KDA_L2NORM_EPS) : 1.f;
+          pred += sm.sdot[j][i][0] * rki * rkj * u[i];
+          o += sm.sdot[j][i][1] * rqj * rki * u[i];
+        }
+        u[j] = sm.sbeta[j] * (to_f32(sm.rv[j][tid]) - pred);
+        o += sm.sdot[j][j][1] * rqj * rkj * u[j];
+        sm.su[j][tid] = u[j];
+        sm.red[0][2 * j][tid] = p.scale * o;
+      }
+    }
+    const bool closed = p.position_states == nullptr;  // only the end state is needed
+    if (closed && tid < DK) {
+      const float gl = sm.sg[Kg - 1][tid];
+      sm.wK[tid] = __expf(gl);
+      for (int j = 0; j < Kg; ++j) {
+        const float rkj = l2norm ? rsqrtf(sm.snrm[j][0] + KDA_L2NORM_EPS) : 1.f;
+        sm.wk[j][tid] = __expf(gl - sm.sg[j][tid]) * sm.sk[j][tid] * rkj;
+      }
+    }
+    __syncthreads();
+    // ---- the state.  With position states: token by token in registers, S_j = Diag(e^{g_j}) S_{j-1}
+    // + k_j u_j^T.  Without: the group's end state in one pass, S = Diag(e^{G_last}) S0 +
+    // sum_j Diag(e^{G_last - G_j}) k_j u_j^T (the same recurrence unrolled; every factor <= 1).
+    if (closed) {
+      float2 u2[KG][2];
+#pragma unroll
+      for (int j = 0; j < KG; ++j) {
+        const float4 u4 = j < Kg ? reinterpret_cast<const float4*>(sm.su[j])[cg] : make_float4(0.f, 0.f, 0.f, 0.f);
+        u2[j][0] = lo2(u4);
+        u2[j][1] = hi2(u4);
+      }
+      const bool last = base + Kg == K;
+#pragma unroll
+      for (int i = 0; i < NP; ++i) {
+        const int r = r0 + RPP * i;
+        const float dk = sm.wK[r];
+        float2 sl = make_float2(s[i].x * dk, s[i].y * dk), sh = make_float2(s[i].z * dk, s[i].w * dk);
+#pragma unroll
+        for (int j = 0; j < KG; ++j) {
+          if (j < Kg) {
+            const float w = sm.wk[j][r];
+            const float2 w2 = make_float2(w, w);
+            sl = ffma2(w2, u2[j][0], sl);
+            sh = ffma2(w2, u2[j][1], sh);
+          }
+        }
+        s[i] = make_float4(sl.x, sl.y, sh.x, sh.y);
+        if (commit && last) __stcs(reinterpret_cast<float4*>(S + (size_t)r * DV) + cg, s[i]);
+      }
+    } else {
+      for (int j = 0; j < Kg; ++j) {
+        const float rkj = l2norm ? rsqrtf(sm.snrm[j][0] + KDA_L2NORM_EPS) : 1.f;
+        const float4 u4 = reinterpret_cast<const float4*>(sm.su[j])[cg];
+        const bool last = base + j == K - 1;
+        const size_t row = ((size_t)n * K + base + j) * p.H + h;
+#pragma unroll
+        for (int i = 0; i < NP; ++i) {
+          const int r = r0 + RPP * i;
+          const float a = sm.sa[j][r], kr = sm.sk[j][r] * rkj;
+          s[i].x = s[i].x * a + kr * u4.x; s[i].y = s[i].y * a + kr * u4.y;
+          s[i].z = s[i].z * a + kr * u4.z; s[i].w = s[i].w * a + kr * u4.w;
+          if (commit && last) __stcs(reinterpret_cast<float4*>(S + (size_t)r * DV) + cg, s[i]);
+        }
+        // the state after this token, for rollback
+        float* P = p.position_states + row * (size_t)(DK * DV);
+#pragma unroll
+        for (int i = 0; i < NP; ++i) __stcs(reinterpret_cast<float4*>(P + (size_t)(r0 + RPP * i) * DV) + cg, s[i]);
+      }
+    }
+    // ---- outputs: warp j takes token j (head-wise RMSNorm over dv, then the sigmoid gate)
+    if (warp < Kg) {
+      const int j = warp;
+      const size_t row = ((size_t)n * K + base + j) * p.H + h;
+      T* op = static_cast<T*>(p.out) + row * DV;
+      const float* so = sm.red[0][2 * j];
+      if (p.gate == nullptr) {
+#pragma unroll
+        for (int c = lane; c < DV; c += 32) op[c] = from_f32<T>(so[c]);
+      } else {
+        float ss = 0.f;
+#pragma unroll
+        for (int c = lane; c < DV; c += 32) ss += so[c] * so[c];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float rr = rsqrtf(ss / (float)DV + p.eps);
+#pragma unroll
+        for (int c = lane; c < DV; c += 32) {
+          const float wj = p.norm_weight ? p.norm_weight[c] : 1.0f;
+          const float gl = to_f32(sm.rgate[j][c]);
+          op[c] = from_f32<T>(so[c] * rr * wj / (1.0f + __expf(-gl)));
+        }
+      }
+    }
+  }
+}
+
 // CTAs of one kernel instance resident on the whole device at once (cached per device; host
 // threads that launch at the same time may each compute it and store the same value)
 template <typename T, int DK, int DV, bool kPre>
@@ -240,7 +591,14 @@ int resident_ctas() {
 template <typename T, int DK, int DV, bool kPre>
 cudaError_t launch_pre(DecodeParams p, int units, cudaStream_t stream) {
   p.ahead = resident_ctas<T, DK, DV, kPre>();
-  decode_kernel<T, DK, DV, kPre><<<units, kThreads, 0, stream>>>(p);
+  if (p.tokens > 1) {
+    const int smem = (int)sizeof(MultiSmem<T, DK, DV>);
+    auto kern = decode_multi_kernel<T, DK, DV, kPre>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<units, kThreads, smem, stream>>>(p);
+  } else
+    decode_kernel<T, DK, DV, kPre><<<units, kThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -19,10 +19,10 @@ constexpr int kPlanMax = 960;  // segments per launch (the plan travels in the k
 
 // Where a unit's start state comes from and where its end state goes.
 enum SegRole : int32_t {
-  kRoleWhole = 0,     // start: initial_state (or 0); end: final_state; writes outputs
+  kRoleWhole = 0,     // start: initial_state (or 0); writes outputs; end: final_state if the segment
+                      //   ends its sequence, else (the first segment of a split sequence) the
+                      //   workspace start-state slot of the next segment
   kRoleLocal = 1,     // split pass 1: start from [0 | I], no outputs; end: workspace slot (S_loc, M)
-  kRoleHead = 2,      // split pass 1, first segment: start from initial_state, no outputs;
-                      //   end state -> workspace start-state slot of the next segment
   kRoleFromWs = 3,    // split pass 2: start from workspace start-state slot; writes outputs;
                       //   end state -> final_state if last segment of its sequence
   kRoleLocalS = 4,    // split pass 1 on the tensor-core kernel: start from 0, no outputs;

@@ -67,6 +67,10 @@ __device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int32_t c0, in
                "r"(c2)
                : "memory");
 }
+// Prefetch of the 128-byte line holding `addr` into L2 (a hint).
+__device__ __forceinline__ void prefetch_l2_line(const void* addr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(addr) : "memory");
+}
 // 3-D tiled load into shared memory, completion counted on `bar` (transaction bytes).
 __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_t* bar, int32_t c0,
                                             int32_t c1, int32_t c2) {

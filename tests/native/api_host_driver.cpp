@@ -124,6 +124,7 @@ void run_and_check(kda_chunk_args a, const std::vector<int32_t>& lens, bool expe
       }
     }
   }
+  for (auto& kv : final_pass) any_split |= kv.second.size() > 1;
   CHECK(any_split == expect_split);
   for (int n = 0; n < N; ++n) {
     auto& v = final_pass[n];

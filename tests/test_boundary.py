@@ -137,11 +137,14 @@ def test_workspace_size_and_check(L):
 
 
 def test_automatic_split_for_long_context(L):
-    # 1 sequence x 16 heads of 1M tokens: 16 units < half of 148 SMs -> split into 9 segments
+    # 1 sequence x 16 heads of 1M tokens: 16 units < half of 148 SMs -> split.  With P segments
+    # the first launch holds 16 x (1 + 2 (P - 2)) units (each first segment in full, S_loc and M
+    # of each middle one) and the last 16 x (P - 1); P = 10 gives 272 units (2 waves of 148) and
+    # 144 (1 wave): 3/10 of the unsplit time, the least for P <= 64.
     rc, n = _ws(L, _args(num_seqs=1, total_tokens=1 << 20, H=16))
     assert rc == B.KDA_OK
     per_slot = 16 * (128 * 128 + 128 * 256) * 4
-    assert (n - 256) % per_slot == 0 and (n - 256) // per_slot == 9
+    assert (n - 256) % per_slot == 0 and (n - 256) // per_slot == 10
 
 
 def _dargs(**kw):

@@ -235,3 +235,25 @@ def test_varlen_neighbour_nan_does_not_leak(path):
         assert torch.isfinite(out[sl]).all() and torch.isfinite(fin[n]).all(), n
         assert rel_l2(host(out[sl]), o_ref) <= TOL_OUT_BF16, n
         assert rel_l2(host(fin[n]), f_ref[0]) <= TOL_STATE_BF16, n
+
+
+_SPLIT_REF = {}
+
+
+@pytest.mark.parametrize("split", [1, 2, 9, 32])
+def test_split_error_against_segment_count(split):
+    """One 65,536-token sequence with slow decay (the state carries across segments), two heads:
+    the same call cut into 1, 2, 9 and 32 segments.  Each segment boundary adds a combine step
+    S_start(q+1) = M_q S_start(q) + S_loc(q) with M_q and S_loc from bf16 tensor-core passes, so
+    the error can grow with the segment count; every count must stay within the tolerances
+    (outputs of the last 4,096 tokens and of the first 4,096, final states)."""
+    T = 65536
+    inp = synth.make_prefill(H=2, dk=128, dv=128, dtype="bf16", seed=39, device="cuda",
+                             lengths=np.array([T]), gate=True, init_state=True, decay_shift=-6.0)
+    if "ref" not in _SPLIT_REF:
+        _SPLIT_REF["ref"] = oracle_full(inp, num_threads=2)
+    o_ref, f_ref = _SPLIT_REF["ref"]
+    out, fin = _run(inp, split=split)
+    for sl in (slice(0, 4096), slice(T - 4096, T)):
+        assert rel_l2(host(out[sl]), o_ref[sl]) <= TOL_OUT_BF16, (split, sl)
+    assert rel_l2(host(fin), f_ref) <= TOL_STATE_BF16, split
