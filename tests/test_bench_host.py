@@ -40,7 +40,7 @@ def test_committed_profiles_carry_a_traffic_line():
         assert "traffic_bytes_per_launch:" in text and "source_sha1:" in text, tag
 
 
-def test_cpu_sample_units_bounded_by_batch_and_cores():
-    assert bench.cpu_sample_units(4, 32, 16) == [(u // 32, u % 32) for u in range(32)]
-    assert len(bench.cpu_sample_units(4, 32, 1000)) == 128  # never more units than the batch has
+def test_cpu_sample_units_cover_the_batch_in_order():
+    # the oracle runs the whole headline batch (about a second on 16 cores)
+    assert bench.cpu_sample_units(4, 32, 16) == [(u // 32, u % 32) for u in range(128)]
     assert bench.cpu_sample_units(1, 2, 0) == [(0, 0), (0, 1)]
