@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         for (int hf = 0; hf < 2; ++hf) {
           tma_prefetch_3d(&maps.k, hf * 64, h, tok);
-          tma_prefetch_3d(&maps.q, hf * 64, h, tok);
+          if (write_out) tma_prefetch_3d(&maps.q, hf * 64, h, tok);
           if (need_v) tma_prefetch_3d(&maps.v, hf * 64, h, tok);
         }
       }
@@ -350,15 +350,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int hf = 0; hf < 2; ++hf) tma_load_3d(sm + OFF_KQ + hf * 16384, &maps.k, &m->full_k, hf * 64, h, tok);
       }
       ik = j;
-      if (lane == 0) okw = wait_bounded(&m->empty_q, par, m, drain_limit, p.error_word) ? 1 : 0;
-      okw = __shfl_sync(0xffffffffu, okw, 0);
-      if (!okw) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&m->full_q, 16384);
-        for (int hf = 0; hf < 2; ++hf)
-          tma_load_3d(sm + OFF_KQ + hf * 16384 + 8192, &maps.q, &m->full_q, hf * 64, h, tok);
+      if (write_out) {  // the split's pass 1 writes no outputs and needs no q
+        if (lane == 0) okw = wait_bounded(&m->empty_q, par, m, drain_limit, p.error_word) ? 1 : 0;
+        okw = __shfl_sync(0xffffffffu, okw, 0);
+        if (!okw) break;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&m->full_q, 16384);
+          for (int hf = 0; hf < 2; ++hf)
+            tma_load_3d(sm + OFF_KQ + hf * 16384 + 8192, &maps.q, &m->full_q, hf * 64, h, tok);
+        }
+        iq = j;
       }
-      iq = j;
       if (!need_v) continue;
       if (lane == 0) okw = wait_bounded(&m->empty_v, par, m, drain_limit, p.error_word) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);
@@ -441,7 +443,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               uchain(tmem + TM_O, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S, 16384, false, 0, id, false),
               uchain(tmem + TM_O + hi, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S + 16384, 16384, false, 0, id,
                      false)};
-          umma_interleaved(c, 8);
+          if (write_out) {
+            umma_interleaved(c, 8);
+          } else {  // the split's pass 1: no outputs, so no O chains
+            const UChain cu[2] = {c[0], c[1]};
+            umma_interleaved(cu, 8);
+          }
         }
         umma_commit(&m->mma);
         ++committed;
@@ -456,7 +463,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                      idesc_bf16_f32(64, 64, 0, 1), true),
               uchain(tmem + TM_S, sm_u + OFF_KH, 8192, false, 0, sm_u + OFF_KL, 8192, false, 0,
                      idesc_bf16_f32(128, 128, 1, 1), true)};
-          umma_interleaved(c, 4);
+          if (write_out) {
+            umma_interleaved(c, 4);
+          } else {
+            const UChain ck[1] = {c[2]};
+            umma_interleaved(ck, 4);
+          }
         }
         umma_commit(&m->mma);
         ++committed;
@@ -688,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------------- decay prep: all bf16 operands
 
       {
-        if (tid == 0 && wait_bounded(&m->full_k, par, m, limit, p.error_word))
+        if (tid == 0 && wait_bounded(&m->full_k, par, m, limit, p.error_word) && write_out)
           wait_bounded(&m->full_q, par, m, limit, p.error_word);
         sync_wg();
         if (*(volatile int32_t*)&m->abort != 0) { ok = false; break; }
@@ -744,10 +756,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           float2 kf[4], qf[4], x[4], ix[4], f[4], fq[4];
           if (t < L) {
             unpack8x2(at16(sm, OFF_KQ + sw128_oct(t, o, 16384)), kf);
-            unpack8x2(at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)), qf);
+            if (write_out) {
+              unpack8x2(at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)), qf);
+            } else {  // no q in the split's pass 1: P and O are not needed
+#pragma unroll
+              for (int c = 0; c < 4; ++c) qf[c] = make_float2(0.f, 0.f);
+            }
             if (l2norm) {  // x / sqrt(|x|^2 + eps)
               const float rk = rsqrtf(m->qkss[0][t] + m->qkss[1][t] + KDA_L2NORM_EPS);
-              const float rq = rsqrtf(m->qkss[0][64 + t] + m->qkss[1][64 + t] + KDA_L2NORM_EPS);
+              const float rq = write_out ? rsqrtf(m->qkss[0][64 + t] + m->qkss[1][64 + t] + KDA_L2NORM_EPS) : 0.f;
 #pragma unroll
               for (int c = 0; c < 4; ++c) {
                 kf[c] = fmul2(kf[c], make_float2(rk, rk));
@@ -829,7 +846,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t v[16];
             tmem_ld16(tl + TM_AP + ap_off(a) + 16 * kb, v);
             tmem_wait_ld();
-            if (mine) {
+            if (mine && (write_out || !isP)) {  // (P only where outputs are written)
               if (!isP) {
 #pragma unroll
                 for (int jj = 0; jj < 16; ++jj) {
@@ -848,7 +865,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (isP && mine) {
+        if (isP && mine && write_out) {
 #pragma unroll
           for (int oc = 0; oc < 8; ++oc)
             if (oc >= 2 * (a + 1)) at16(sm, OFF_P + sw128_oct(t, oc, 8192)) = make_uint4(0u, 0u, 0u, 0u);
@@ -1038,7 +1055,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (!r || !next_ok) { ok = false; break; }
       }
-      if (tid == 0) mbar_arrive(&m->empty_q);  // the q rows (e^{gamma} q in place) consumed
+      if (tid == 0 && write_out) mbar_arrive(&m->empty_q);  // the q rows (e^{gamma} q in place) consumed
 
       // ---------------------------------------------------------------- U -> bf16 (same lane split as -W)
       {

@@ -92,7 +92,9 @@ def test_no_commit_leaves_state_unchanged():
 def test_verify_then_roll_back_or_commit_prefix():
     """Speculative decoding: verify K = 4 drafts without committing; accept m = 2.  Taking the
     position-1 state and re-running the 2 accepted tokens with commit give the same state, and
-    both continue like the oracle that saw only the accepted tokens."""
+    both continue like the oracle that saw only the accepted tokens.  (The position states come
+    from the token-by-token update, the committed state from the same recurrence unrolled over
+    the group, so they agree to fp32 rounding rather than bit for bit.)"""
     N, H, K, m = 6, 2, 4, 2
     state = synth.make_states(slots=N, H=H, dk=128, dv=128, seed=64, device="cuda")
     s64 = state.double().cpu().numpy()
@@ -102,7 +104,7 @@ def test_verify_then_roll_back_or_commit_prefix():
     rolled = pos[:, m - 1].contiguous()
     acc = {n: x[:, :m].contiguous() for n, x in t.items()}
     _run(acc, state)  # commit the accepted prefix
-    torch.testing.assert_close(state, rolled, rtol=0, atol=0)
+    torch.testing.assert_close(state, rolled, rtol=1e-5, atol=1e-6)
     _, _ = _oracle_steps(acc, s64, None)
     assert rel_l2(state.cpu().numpy(), s64) <= TOL_STATE_BF16
     nxt = _tokens(N, 1, H, 128, 128, "bf16", seed=66)
