@@ -240,9 +240,8 @@ __device__ __forceinline__ void umma_interleaved(const UChain (&c)[NC], int kste
   }
 }
 
-template <bool kPre>
-__global__ void __launch_bounds__(kThreads, 1)
-    chunk_tc_kernel(const __grid_constant__ Plan plan, const __grid_constant__ TcMaps maps, const ChunkParams p) {
+template <bool kPre, bool kOut>
+__device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& maps, const ChunkParams& p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-byte aligned base (swizzle atoms), offset by pointer arithmetic on the __shared__ array so
   // that every access through sm stays a shared-memory access
@@ -263,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint64_t drain_limit = 2000000000ull;
   const int nchunks = (seg.len + C - 1) / C;
   const bool need_v = seg.role != kRoleLocalM;  // the transition pass runs with values = 0
-  const bool write_out = (seg.role == kRoleWhole || seg.role == kRoleFromWs);
+  constexpr bool write_out = kOut;
   const bool stage_gate = write_out && has_gate;  // the epilogue needs the chunk's gate logits
 
   if (tid == 0) {
@@ -1131,6 +1130,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
+}
+
+// The body is compiled twice: with outputs, and without them for the split's pass-1 roles
+// (no q, no P, no Q.S or P.U chains, no epilogue). A CTA's role is uniform, so each CTA runs one
+// copy, and the output copy carries no run-time tests of the role.
+template <bool kPre>
+__global__ void __launch_bounds__(kThreads, 1)
+    chunk_tc_kernel(const __grid_constant__ Plan plan, const __grid_constant__ TcMaps maps, const ChunkParams p) {
+  const int role = plan.seg[blockIdx.x / plan.H].role;
+  if (role == kRoleWhole || role == kRoleFromWs)
+    chunk_tc_body<kPre, true>(plan, maps, p);
+  else
+    chunk_tc_body<kPre, false>(plan, maps, p);
 }
 
 // ------------------------------------------------------------------ host side
