@@ -84,17 +84,17 @@ bool uses_tensor_cores(const kda_chunk_args* a) {
 int64_t waves(int64_t units) { return (units + kPlanSMs - 1) / kPlanSMs; }
 
 // Automatic segment count for `busy` (sequence, head) units of one long length: the split runs
-// launch A (each sequence's first segment in full, and pass 1 of the middle segments: two units
-// each on the tensor cores, S_loc and the transition M; one augmented unit on the CUDA cores,
-// launched on its own), the combine, and launch B (the other segments from their start states).
-// Every unit of a launch takes the time of one segment, so the call takes about
+// launch A (each sequence's first segment in full, and pass 1 of the middle segments: one unit
+// on the augmented state [S_loc | M] each, in the same launch on the tensor cores and in a
+// launch of its own on the CUDA cores), the combine, and launch B (the other segments from their
+// start states).  Every unit of a launch takes the time of one segment, so the call takes about
 // (waves of A + waves of B) / P of the unsplit time; the P with the least is taken, if it
 // saves at least a fifth.
 int32_t auto_segments(int64_t busy, bool tc) {
   int32_t best = 1;
   double best_t = 0.8;
   for (int32_t P = 2; P <= 64; ++P) {
-    const int64_t w = tc ? waves(busy * (1 + 2 * (int64_t)(P - 2)))
+    const int64_t w = tc ? waves(busy * (int64_t)(P - 1))
                          : waves(busy) + (P > 2 ? waves(busy * (int64_t)(P - 2)) : 0);
     const double t = (double)(w + waves(busy * (int64_t)(P - 1))) / P;
     if (t < best_t - 1e-9) {
@@ -275,8 +275,8 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
   // Launch A: every unsplit sequence, and the first segment of each split sequence, in full from
   // its initial state (outputs, snapshots; a first segment also leaves its end state in the
   // workspace as the second segment's start state); with them pass 1 of the middle segments
-  // (local state from zero and the transition matrix; on the CUDA cores as one augmented unit,
-  // launched on its own because its kernel differs).  Then the combine, then launch B: the
+  // (local state from zero and the transition matrix, as one unit on the augmented state; on the
+  // CUDA cores launched on its own because its kernel differs).  Then the combine, then launch B: the
   // remaining segments of the split sequences from their start states.
   std::vector<Seg> first, local, rest;
   std::vector<int64_t> snap_base;
@@ -302,9 +302,8 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
         continue;
       }
       if (q < np - 1) {
-        if (use_tc) {  // S_loc and M as two plain-state units of the tensor-core kernel
-          first.push_back(make_seg(t0, len, sp.seq, kRoleLocalS, b + q, 0));
-          first.push_back(make_seg(t0, len, sp.seq, kRoleLocalM, b + q, 0));
+        if (use_tc) {  // [S_loc | M] beside the first segments, in the same launch
+          first.push_back(make_seg(t0, len, sp.seq, kRoleLocal, b + q, 0));
         } else {
           local.push_back(make_seg(t0, len, sp.seq, kRoleLocal, b + q, 0));
         }

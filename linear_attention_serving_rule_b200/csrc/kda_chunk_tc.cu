@@ -42,6 +42,11 @@
 // a warp's 32 lanes read 16 rows x 2 column halves and every lane takes part in the read-outs.
 // O keeps its own columns so that a chunk's epilogue can run beside the next chunk's UMMAs.
 //
+// The split's pass 1 (a middle segment's local state and transition matrix, no outputs) runs a
+// second copy of the same body on the augmented state [S | M]: no q tile, no P, and the output
+// chains replaced by M's (U_M = -W M, M += Kh^T U_M); its TMEM and shared-memory map is given
+// beside the layout constants below.
+//
 // Every wait is bounded (%globaltimer): on expiry the kernel records KDA_ERR_TIMEOUT, stops
 // issuing work, drains its own in-flight TMA and UMMA operations (bounded again), frees TMEM
 // and returns.
@@ -84,6 +89,16 @@ constexpr int LDT = 68;
 constexpr uint32_t OFF_TF = OFF_KC + 64 * LDF * 4;
 
 constexpr uint32_t TM_S = 0, TM_AP = 128, TM_WU = 288, TM_O = 416;
+// The split's pass 1 runs on the augmented state [S | M] (S from 0 with the values, M from I
+// with values 0, so it ends as the segment's transition matrix) and writes no outputs. Its TMEM:
+// [0,128) S, [128,256) M, [256,416) A|P; once A is read out, W|U' over [256,384) and U_M = -W M
+// in [384,448). Its shared memory reuses what the outputs would take: M's bf16 copy (the B
+// operand of -W M) in the gate buffer and in the second column block of the [k; q] tile, which is
+// free once the Gram is done; U_M in bf16 over T' and P, free once the W|U' UMMAs are done.
+constexpr uint32_t TM_M = 128, TM_AP_AUG = 256, TM_WU_AUG = 256, TM_UM = 384;
+constexpr uint32_t OFF_MC0 = OFF_GATE, OFF_MC1 = OFF_KL + 16384, OFF_UM = OFF_TP;
+static_assert(OFF_TP + 8192 == OFF_P, "U_M's two column blocks sit over T' and P, 8 KB apart");
+static_assert(OFF_MC0 % 1024 == 0 && OFF_MC1 % 1024 == 0, "swizzle atoms need 1024-byte alignment");
 
 // The column operands Kc_0..Kc_3 (16(a+1) rows each) are stacked into one 160-row K-major tile
 // (two 64-column blocks of 160 x 128 bytes); Kc_a starts at row ap_off(a), which is also the
@@ -261,7 +276,7 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
   const uint64_t limit = (p.flags & KDA_FLAG_TEST_FORCE_TIMEOUT) ? 0ull : 2000000000ull;  // 2 s
   const uint64_t drain_limit = 2000000000ull;
   const int nchunks = (seg.len + C - 1) / C;
-  const bool need_v = seg.role != kRoleLocalM;  // the transition pass runs with values = 0
+  constexpr uint32_t tm_ap = kOut ? TM_AP : TM_AP_AUG, tm_wu = kOut ? TM_WU : TM_WU_AUG;
   constexpr bool write_out = kOut;
   const bool stage_gate = write_out && has_gate;  // the epilogue needs the chunk's gate logits
 
@@ -313,7 +328,7 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
         for (int hf = 0; hf < 2; ++hf) {
           tma_prefetch_3d(&maps.k, hf * 64, h, tok);
           if (write_out) tma_prefetch_3d(&maps.q, hf * 64, h, tok);
-          if (need_v) tma_prefetch_3d(&maps.v, hf * 64, h, tok);
+          tma_prefetch_3d(&maps.v, hf * 64, h, tok);
         }
       }
       int okw = 1;
@@ -360,7 +375,6 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
         }
         iq = j;
       }
-      if (!need_v) continue;
       if (lane == 0) okw = wait_bounded(&m->empty_v, par, m, drain_limit, p.error_word) ? 1 : 0;
       okw = __shfl_sync(0xffffffffu, okw, 0);
       if (!okw) break;
@@ -403,7 +417,7 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
           const uint32_t id = idesc_bf16_f32(128, KC_ROWS, 0, 0);
 #pragma unroll 1
           for (int k = 0; k < 8; ++k)  // (a rolled loop: each step waits ~180 cycles anyway)
-            umma_bf16(tmem + TM_AP, a0 + (((k >> 2) * 16384u + (k & 3) * 32u) >> 4),
+            umma_bf16(tmem + tm_ap, a0 + (((k >> 2) * 16384u + (k & 3) * 32u) >> 4),
                       b0 + (((k >> 2) * KC_BLK + (k & 3) * 32u) >> 4), id, k > 0 ? 1u : 0u);
         }
         umma_commit(&m->mma);
@@ -412,61 +426,63 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
         // [352,416); one N=128 UMMA per half, whose B operand is [e^g k block | v block] -- two MN
         // atoms (OFF_V - OFF_KQ) and (OFF_V + 8192 - OFF_KQ - 16384) bytes apart
         if (!wait_bounded(&m->ops, (oph++) & 1u, m, limit, p.error_word)) break;
-        if (need_v && !wait_bounded(&m->full_v, par, m, limit, p.error_word)) break;
+        if (!wait_bounded(&m->full_v, par, m, limit, p.error_word)) break;
         tc_fence_after();
-        if (need_v) {
+        {
           const uint32_t id = idesc_bf16_f32(64, 128, 0, 1);
           const UChain c[2] = {
-              uchain(tmem + TM_WU, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ, OFF_V - OFF_KQ, false, 0, id, false),
-              uchain(tmem + TM_WU + hi, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ + 16384,
+              uchain(tmem + tm_wu, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ, OFF_V - OFF_KQ, false, 0, id, false),
+              uchain(tmem + tm_wu + hi, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ + 16384,
                      OFF_V + 8192 - OFF_KQ - 16384, false, 0, id, false)};
-          umma_interleaved(c, 4);
-        } else {
-          const uint32_t id = idesc_bf16_f32(64, 64, 0, 1);
-          const UChain c[2] = {
-              uchain(tmem + TM_WU, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ, 16384, false, 0, id, false),
-              uchain(tmem + TM_WU + hi, sm_u + OFF_TP, 16, true, 0, sm_u + OFF_KQ + 16384, 16384, false, 0, id, false)};
           umma_interleaved(c, 4);
         }
         umma_commit(&m->mma);
         ++committed;
-        // U = U' - W S0 ; O = Qt S0
+        // U = U' - W S0 ; O = Qt S0  (pass 1: U = U' - W S0 ; U_M = -W M0)
         if (!wait_bounded(&m->ops, (oph++) & 1u, m, limit, p.error_word)) break;
         tc_fence_after();
         {
           const uint32_t id = idesc_bf16_f32(64, 64, 0, 1);
-          const UChain c[4] = {
-              uchain(tmem + TM_WU + 64, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S, 16384, false, 0, id, need_v),
-              uchain(tmem + TM_WU + 64 + hi, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S + 16384, 16384, false, 0, id,
-                     need_v),
-              uchain(tmem + TM_O, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S, 16384, false, 0, id, false),
-              uchain(tmem + TM_O + hi, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S + 16384, 16384, false, 0, id,
-                     false)};
-          if (write_out) {
+          const UChain cu0 = uchain(tmem + tm_wu + 64, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S, 16384, false, 0,
+                                    id, true);
+          const UChain cu1 = uchain(tmem + tm_wu + 64 + hi, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_S + 16384,
+                                    16384, false, 0, id, true);
+          if (kOut) {
+            const UChain c[4] = {
+                cu0, cu1,
+                uchain(tmem + TM_O, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S, 16384, false, 0, id, false),
+                uchain(tmem + TM_O + hi, sm_u + OFF_KQ + 8192, 16, true, 16384, sm_u + OFF_S + 16384, 16384, false, 0,
+                       id, false)};
             umma_interleaved(c, 8);
-          } else {  // the split's pass 1: no outputs, so no O chains
-            const UChain cu[2] = {c[0], c[1]};
-            umma_interleaved(cu, 8);
+          } else {
+            const UChain c[4] = {
+                cu0, cu1,
+                uchain(tmem + TM_UM, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_MC0, 16384, false, 0, id, false),
+                uchain(tmem + TM_UM + hi, sm_u + OFF_KL, 16, true, 8192, sm_u + OFF_MC1, 16384, false, 0, id, false)};
+            umma_interleaved(c, 8);
           }
         }
         umma_commit(&m->mma);
         ++committed;
-        // O += P U ; S += Kh^T U
+        // O += P U ; S += Kh^T U  (pass 1: S += Kh^T U ; M += Kh^T U_M)
         if (!wait_bounded(&m->ops, (oph++) & 1u, m, limit, p.error_word)) break;
         tc_fence_after();
         {
-          const UChain c[3] = {
-              uchain(tmem + TM_O, sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL, 8192, false, 0, idesc_bf16_f32(64, 64, 0, 1),
-                     true),
-              uchain(tmem + TM_O + hi, sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL + 8192, 8192, false, 0,
-                     idesc_bf16_f32(64, 64, 0, 1), true),
-              uchain(tmem + TM_S, sm_u + OFF_KH, 8192, false, 0, sm_u + OFF_KL, 8192, false, 0,
-                     idesc_bf16_f32(128, 128, 1, 1), true)};
-          if (write_out) {
+          const UChain cs = uchain(tmem + TM_S, sm_u + OFF_KH, 8192, false, 0, sm_u + OFF_KL, 8192, false, 0,
+                                   idesc_bf16_f32(128, 128, 1, 1), true);
+          if (kOut) {
+            const UChain c[3] = {
+                uchain(tmem + TM_O, sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL, 8192, false, 0,
+                       idesc_bf16_f32(64, 64, 0, 1), true),
+                uchain(tmem + TM_O + hi, sm_u + OFF_P, 16, true, 0, sm_u + OFF_KL + 8192, 8192, false, 0,
+                       idesc_bf16_f32(64, 64, 0, 1), true),
+                cs};
             umma_interleaved(c, 4);
           } else {
-            const UChain ck[1] = {c[2]};
-            umma_interleaved(ck, 4);
+            const UChain c[2] = {
+                cs, uchain(tmem + TM_M, sm_u + OFF_KH, 8192, false, 0, sm_u + OFF_UM, 8192, false, 0,
+                           idesc_bf16_f32(128, 128, 1, 1), true)};
+            umma_interleaved(c, 4);
           }
         }
         umma_commit(&m->mma);
@@ -516,21 +532,21 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
       } else if (seg.role == kRoleFromWs) {
         src = p.ws_state + ((size_t)seg.slot * H + h) * unit_state;
       }
-      const bool ident = seg.role == kRoleLocalM;  // transition pass: start from I
 #pragma unroll
       for (int hb = 0; hb < 2; ++hb) {
         const int c0 = wg * 64 + hb * 32;
         uint32_t v[32];
+        if (!kOut) {  // pass 1: M = I (its bf16 copy is made per chunk, beside the W|U' UMMAs)
+#pragma unroll
+          for (int jj = 0; jj < 32; ++jj) v[jj] = __float_as_uint(c0 + jj == row ? 1.f : 0.f);
+          tmem_st32(tl + TM_M + c0, v);
+        }
 #pragma unroll
         for (int jj = 0; jj < 32; jj += 4) {
           float4 x = src ? *reinterpret_cast<const float4*>(src + (size_t)row * DV + c0 + jj)
                          : make_float4(0.f, 0.f, 0.f, 0.f);
           v[jj] = __float_as_uint(x.x); v[jj + 1] = __float_as_uint(x.y);
           v[jj + 2] = __float_as_uint(x.z); v[jj + 3] = __float_as_uint(x.w);
-        }
-        if (ident) {
-#pragma unroll
-          for (int jj = 0; jj < 32; ++jj) v[jj] = __float_as_uint(c0 + jj == row ? 1.f : 0.f);
         }
         tmem_st32(tl + TM_S + c0, v);
 #pragma unroll
@@ -782,12 +798,12 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
 #pragma unroll
           for (int c = 0; c < 4; ++c) { f[c] = fmul2(kf[c], x[c]); fq[c] = fmul2(qf[c], x[c]); }
           at16(sm, OFF_KL + sw128_oct(t, o, 16384)) = pack8x2(f);
-          at16(sm, OFF_KL + sw128_oct(64 + t, o, 16384)) = pack8x2(fq);
+          if (write_out) at16(sm, OFF_KL + sw128_oct(64 + t, o, 16384)) = pack8x2(fq);
           // e^{gamma} k and e^{gamma} q, in place over the raw tiles (this thread's own elements)
 #pragma unroll
           for (int c = 0; c < 4; ++c) { f[c] = fmul2(f[c], Eb2[c]); fq[c] = fmul2(fq[c], Eb2[c]); }
           at16(sm, OFF_KQ + sw128_oct(t, o, 16384)) = pack8x2(f);
-          at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)) = pack8x2(fq);
+          if (write_out) at16(sm, OFF_KQ + sw128_oct(64 + t, o, 16384)) = pack8x2(fq);
           // Kc_a = k e^{r_a - gamma_t}: k ix for a = b, then k ix se_b se_{b+1} ... se_{a-1};
           // the last one (a = 3) times se_3 is e^{gamma_C - gamma_t} k, the state-carry operand
 #pragma unroll
@@ -843,7 +859,7 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
         for (int kb = 0; kb < 4; ++kb) {
           if (kb <= a) {
             uint32_t v[16];
-            tmem_ld16(tl + TM_AP + ap_off(a) + 16 * kb, v);
+            tmem_ld16(tl + tm_ap + ap_off(a) + 16 * kb, v);
             tmem_wait_ld();
             if (mine && (write_out || !isP)) {  // (P only where outputs are written)
               if (!isP) {
@@ -985,7 +1001,7 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
       // A partial last chunk: the v tile's rows t >= L hold the next sequence's tokens (or the
       // zero fill past the tensor).  T' has zero columns there (beta = 0), but 0 * Inf or NaN is
       // NaN, so the rows are cleared: a sequence must not see its neighbour's values at all.
-      if (need_v && L < C) {
+      if (L < C) {
         if (!wg_wait(&m->full_v, par)) { ok = false; break; }
         for (int idx = tid; idx < (C - L) * 16; idx += kCompute) {
           const int t = L + (idx >> 4), c16 = idx & 15;  // a row's 16-byte chunks, either block
@@ -994,6 +1010,19 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
       }
       ops_arrive();  // ---------------------------------------------- UMMA: W = T' Kt, U' = T' V
       if (write_out && j > 0) epilogue_b(L_prev, tok_prev);  // in the shadow of the W|U' UMMAs
+      if (!kOut) {  // pass 1: M's bf16 copy, column half wg of this warp's rows (the Gram is done)
+        uint32_t v[64];
+        tmem_ld32(tl + TM_M + 64 * wg, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+        tmem_ld32(tl + TM_M + 64 * wg + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+        tmem_wait_ld();
+#pragma unroll
+        for (int oc = 0; oc < 8; ++oc) {
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
+          at16(sm, (wg ? OFF_MC1 : OFF_MC0) + sw128_oct(row, oc, 16384)) = pack8(f);
+        }
+      }
       {
         const bool r = wg_wait(&m->mma, mph & 1u);
         ++mph;
@@ -1001,7 +1030,7 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
         if (!r) { ok = false; break; }
       }
       if (tid == 0) {  // v and the k rows (e^{gamma} k in place) consumed
-        if (need_v) mbar_arrive(&m->empty_v);
+        mbar_arrive(&m->empty_v);
         mbar_arrive(&m->empty_k);
         if (stage_gate && j > 0) mbar_arrive(&m->empty_gate);  // chunk j - 1's epilogue is done
       }
@@ -1012,7 +1041,7 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
         const int t = 16 * q4 + (lane & 15);
         const int c0 = (lane >> 4) * 64 + wg * 32;
         uint32_t v[32];
-        tmem_ld32(tl + TM_WU + 32 * wg, v);
+        tmem_ld32(tl + tm_wu + 32 * wg, v);
         tmem_wait_ld();
 #pragma unroll
         for (int oc = 0; oc < 4; ++oc) {
@@ -1029,14 +1058,14 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
       {
         const float ec = m->ec[row];
 #pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-          const int c0 = 64 * wg + 32 * hb;
+        for (int hb = 0; hb < (kOut ? 2 : 4); ++hb) {  // (pass 1: the rows of M too)
+          const uint32_t c0 = (hb < 2 ? TM_S : TM_M) + 64 * wg + 32 * (hb & 1);
           uint32_t v[32];
-          tmem_ld32(tl + TM_S + c0, v);
+          tmem_ld32(tl + c0, v);
           tmem_wait_ld();
 #pragma unroll
           for (int jj = 0; jj < 32; ++jj) v[jj] = __float_as_uint(__uint_as_float(v[jj]) * ec);
-          tmem_st32(tl + TM_S + c0, v);
+          tmem_st32(tl + c0, v);
         }
         tmem_wait_st();
       }
@@ -1061,7 +1090,7 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
         const int t = 16 * q4 + (lane & 15);
         const int c0 = (lane >> 4) * 64 + wg * 32;
         uint32_t v[32];
-        tmem_ld32(tl + TM_WU + 64 + 32 * wg, v);
+        tmem_ld32(tl + tm_wu + 64 + 32 * wg, v);
         tmem_wait_ld();
 #pragma unroll
         for (int oc = 0; oc < 4; ++oc) {
@@ -1069,6 +1098,17 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
 #pragma unroll
           for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
           at16(sm, OFF_KL + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
+        }
+        if (!kOut) {  // pass 1: U_M over T' and P (the W|U' UMMAs that read T' are done)
+          tmem_ld32(tl + TM_UM + 32 * wg, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int oc = 0; oc < 4; ++oc) {
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * oc + e]);
+            at16(sm, OFF_UM + sw128_oct(t, (c0 >> 3) + oc, 8192)) = pack8(f);
+          }
         }
       }
       ops_arrive();  // ---------------------------------------------- UMMA: O += P U ; S += Kh^T U
@@ -1101,24 +1141,25 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
         }
       }
       size_t ld = DV;
-      if (seg.role == kRoleLocalS || seg.role == kRoleLocalM) {  // (S_loc | M) block, row stride dv + dk
+      if (!kOut) {  // pass 1: the (S_loc | M) block of the slot, row stride dv + dk
         ld = DV + DK;
-        dst = p.ws_local + ((size_t)seg.slot * H + h) * (size_t)DK * ld + (seg.role == kRoleLocalM ? DV : 0);
+        dst = p.ws_local + ((size_t)seg.slot * H + h) * (size_t)DK * ld;
       }
-      float* sdst = nchunks > 0 ? snap_dst(seg.len) : nullptr;  // a snapshot boundary at the segment end
+      float* sdst = kOut && nchunks > 0 ? snap_dst(seg.len) : nullptr;  // a snapshot boundary at the segment end
       if (dst || sdst) {
 #pragma unroll
-        for (int hb = 0; hb < 2; ++hb) {
-          const int c0 = wg * 64 + hb * 32;
+        for (int hb = 0; hb < (kOut ? 2 : 4); ++hb) {
+          const int c0 = wg * 64 + (hb & 1) * 32;  // column of S (hb < 2) or of M
           uint32_t v[32];
-          tmem_ld32(tl + TM_S + c0, v);
+          tmem_ld32(tl + (hb < 2 ? TM_S : TM_M) + c0, v);
           tmem_wait_ld();
+          const int cd = (hb < 2 ? 0 : DV) + c0;
 #pragma unroll
           for (int jj = 0; jj < 32; jj += 4) {
             const float4 x = make_float4(__uint_as_float(v[jj]), __uint_as_float(v[jj + 1]),
                                          __uint_as_float(v[jj + 2]), __uint_as_float(v[jj + 3]));
-            if (dst) *reinterpret_cast<float4*>(dst + (size_t)row * ld + c0 + jj) = x;
-            if (sdst) *reinterpret_cast<float4*>(sdst + (size_t)row * DV + c0 + jj) = x;
+            if (dst) *reinterpret_cast<float4*>(dst + (size_t)row * ld + cd + jj) = x;
+            if (sdst && hb < 2) *reinterpret_cast<float4*>(sdst + (size_t)row * DV + c0 + jj) = x;
           }
         }
       }

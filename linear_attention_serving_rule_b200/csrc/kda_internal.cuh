@@ -22,14 +22,10 @@ enum SegRole : int32_t {
   kRoleWhole = 0,     // start: initial_state (or 0); writes outputs; end: final_state if the segment
                       //   ends its sequence, else (the first segment of a split sequence) the
                       //   workspace start-state slot of the next segment
-  kRoleLocal = 1,     // split pass 1: start from [0 | I], no outputs; end: workspace slot (S_loc, M)
+  kRoleLocal = 1,     // split pass 1: start from [0 | I] (the augmented state [S | M], values
+                      //   augmented by zeros), no outputs; end: workspace slot (S_loc | M)
   kRoleFromWs = 3,    // split pass 2: start from workspace start-state slot; writes outputs;
                       //   end state -> final_state if last segment of its sequence
-  kRoleLocalS = 4,    // split pass 1 on the tensor-core kernel: start from 0, no outputs;
-                      //   end state -> columns [0, dv) of the slot's (S_loc | M) block
-  kRoleLocalM = 5,    // split pass 1 on the tensor-core kernel: start from I with values taken
-                      //   as zero (so the end state is the segment's transition M), no outputs;
-                      //   end state -> columns [dv, dv + dk) of the slot's (S_loc | M) block
 };
 
 struct Seg {
