@@ -83,20 +83,21 @@ bool uses_tensor_cores(const kda_chunk_args* a) {
 
 int64_t waves(int64_t units) { return (units + kPlanSMs - 1) / kPlanSMs; }
 
-// Automatic segment count for `busy` (sequence, head) units of one long length: the split runs
-// launch A (each sequence's first segment in full, and pass 1 of the middle segments: one unit
-// on the augmented state [S_loc | M] each, in the same launch on the tensor cores and in a
-// launch of its own on the CUDA cores), the combine, and launch B (the other segments from their
-// start states).  Every unit of a launch takes the time of one segment, so the call takes about
-// (waves of A + waves of B) / P of the unsplit time; the P with the least is taken, if it
-// saves at least a fifth.
-int32_t auto_segments(int64_t busy, bool tc) {
+// Automatic segment count for `busy` (sequence, head) units whose longest sequence has `chunks`
+// 64-token chunks: the split runs launch A (pass 1 of every segment but the last: one unit on the
+// augmented state [S_loc | M] each), the combine, and launch B (every segment from its start
+// state, with outputs).  In chunk times of one unit, a launch takes its waves times the chunks of
+// a segment, and the combine about kCombineStep per segment boundary it chains (one dk x dk by
+// dk x dv product per (sequence, head) in fp32: measured ~37 us against ~9 us per chunk).  The P
+// with the least time is taken, if it saves at least a fifth of the unsplit time.
+constexpr int64_t kCombineStep = 4;
+int32_t auto_segments(int64_t busy, int64_t chunks) {
   int32_t best = 1;
-  double best_t = 0.8;
+  double best_t = 0.8 * (double)chunks;
   for (int32_t P = 2; P <= 64; ++P) {
-    const int64_t w = tc ? waves(busy * (int64_t)(P - 1))
-                         : waves(busy) + (P > 2 ? waves(busy * (int64_t)(P - 2)) : 0);
-    const double t = (double)(w + waves(busy * (int64_t)(P - 1))) / P;
+    const int64_t seg_chunks = (chunks + P - 1) / P;
+    const double t = (double)((waves(busy * (int64_t)(P - 1)) + waves(busy * (int64_t)P)) * seg_chunks +
+                              kCombineStep * (P - 1));
     if (t < best_t - 1e-9) {
       best_t = t;
       best = P;
@@ -121,12 +122,15 @@ Layout make_layout(const kda_chunk_args* a) {
     L.seqs[n] = {t0, len, n};
   }
   // Sequence split: automatic when the (sequence, head) units cannot fill half the GPU.
-  int64_t busy = 0;
-  for (const auto& s : L.seqs) busy += (s.len > 0) ? a->H : 0;
+  int64_t busy = 0, max_len = 0;
+  for (const auto& s : L.seqs) {
+    busy += (s.len > 0) ? a->H : 0;
+    max_len = std::max<int64_t>(max_len, s.len);
+  }
   int32_t P = 1;
   bool auto_mode = a->split_segments == 0;
   if (auto_mode) {
-    if (busy > 0 && busy * 2 <= kPlanSMs) P = auto_segments(busy, uses_tensor_cores(a));
+    if (busy > 0 && busy * 2 <= kPlanSMs) P = auto_segments(busy, (max_len + 63) / 64);
   } else {
     P = a->split_segments;
   }
@@ -272,13 +276,14 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
 
   const bool use_tc = uses_tensor_cores(a);
 
-  // Launch A: every unsplit sequence, and the first segment of each split sequence, in full from
-  // its initial state (outputs, snapshots; a first segment also leaves its end state in the
-  // workspace as the second segment's start state); with them pass 1 of the middle segments
-  // (local state from zero and the transition matrix, as one unit on the augmented state; on the
-  // CUDA cores launched on its own because its kernel differs).  Then the combine, then launch B: the
-  // remaining segments of the split sequences from their start states.
-  std::vector<Seg> first, local, rest;
+  // Launch A: pass 1 of every segment of a split sequence but the last (local state from zero and
+  // the transition matrix, one unit on the augmented state each).  Then the combine, which chains
+  // the start states from the initial state.  Then launch B: every segment of the split sequences
+  // from its start state, and every unsplit sequence from its initial state (outputs, snapshots,
+  // final states).  Each launch runs one kind of unit only: on the tensor cores a launch that
+  // mixed the pass-1 body with the output body measured some of its CTAs 1.7x slower than either
+  // kind alone.
+  std::vector<Seg> local, rest;
   std::vector<int64_t> snap_base;
   if (a->snapshots) snap_base = snapshot_bases(L, a->snapshot_interval, nullptr);
   // segments that carry the true state write the snapshots inside them
@@ -290,36 +295,26 @@ extern "C" kda_status kda_chunk_fwd(const kda_chunk_args* a, void* cuda_stream) 
     const SeqSpan& sp = L.seqs[n];
     const int32_t np = L.nseg[n];
     if (np == 1) {
-      first.push_back(with_snap(make_seg(sp.tok0, sp.len, sp.seq, kRoleWhole, -1, 1), n));
+      rest.push_back(with_snap(make_seg(sp.tok0, sp.len, sp.seq, kRoleWhole, -1, 1), n));
       continue;
     }
     const int32_t sl = L.seglen[n], b = L.slot0[n];
     for (int32_t q = 0; q < np; ++q) {
       const int32_t t0 = sp.tok0 + q * sl;
       const int32_t len = std::min(sl, sp.len - q * sl);
-      if (q == 0) {  // in full; its end state -> start-state slot b + 1
-        first.push_back(with_snap(make_seg(t0, len, sp.seq, kRoleWhole, b, 0), n));
-        continue;
-      }
-      if (q < np - 1) {
-        if (use_tc) {  // [S_loc | M] beside the first segments, in the same launch
-          first.push_back(make_seg(t0, len, sp.seq, kRoleLocal, b + q, 0));
-        } else {
-          local.push_back(make_seg(t0, len, sp.seq, kRoleLocal, b + q, 0));
-        }
-      }
+      if (q < np - 1) local.push_back(make_seg(t0, len, sp.seq, kRoleLocal, b + q, 0));
       rest.push_back(with_snap(make_seg(t0, len, sp.seq, kRoleFromWs, b + q, q == np - 1 ? 1 : 0), n));
     }
   }
-  cudaError_t e = run_segments(first, p, a->dtype, use_tc, stream);
-  if (e == cudaSuccess && !local.empty()) e = run_segments(local, p, a->dtype, use_tc, stream);
+  cudaError_t e = local.empty() ? cudaSuccess : run_segments(local, p, a->dtype, use_tc, stream);
   if (e == cudaSuccess && L.any_split) {
-    // combine: S_start(q+1) = M_q S_start(q) + S_loc(q), sequential over q per (sequence, head)
+    // combine: S_start(0) = the initial state, S_start(q+1) = M_q S_start(q) + S_loc(q),
+    // sequential over q per (sequence, head)
     static thread_local Plan plan;
     plan.H = a->H;
     plan.n_seg = 0;
     for (int32_t n = 0; n < a->num_seqs && e == cudaSuccess; ++n) {
-      if (L.nseg[n] <= 2) continue;
+      if (L.nseg[n] <= 1) continue;
       plan.seg[plan.n_seg++] = make_seg(L.seqs[n].tok0, L.nseg[n], L.seqs[n].seq, kRoleLocal, L.slot0[n], 0);
       if (plan.n_seg == kPlanMax) {
         e = launch_split_combine(plan, p, 0, stream);

@@ -286,11 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* dst = nullptr;
   int ld = DV;
   if (seg.role == kRoleWhole || seg.role == kRoleFromWs) {
-    if (seg.last) {
-      if (p.final_state) dst = p.final_state + ((size_t)seg.seq * H + h) * (size_t)(DK * DV);
-    } else if (seg.role == kRoleWhole) {  // first segment of a split sequence: the next one's start
-      dst = p.ws_state + ((size_t)(seg.slot + 1) * H + h) * (size_t)(DK * DV);
-    }
+    if (seg.last && p.final_state) dst = p.final_state + ((size_t)seg.seq * H + h) * (size_t)(DK * DV);
   } else {  // kRoleLocal: [S_loc | M]
     dst = p.ws_local + ((size_t)seg.slot * H + h) * (size_t)(DK * (DV + DK));
     ld = DV + DK;

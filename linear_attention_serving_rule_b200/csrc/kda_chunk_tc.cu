@@ -855,25 +855,35 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
         const int a = 2 * (q4 & 1) + wg;  // the sub-tile whose columns this warp loads
         const bool mine = (t >> 4) == a;
         const float bt = beta[t];
+        // the warp's column blocks two at a time: both loads in flight, then one wait
 #pragma unroll
-        for (int kb = 0; kb < 4; ++kb) {
-          if (kb <= a) {
-            uint32_t v[16];
-            tmem_ld16(tl + tm_ap + ap_off(a) + 16 * kb, v);
-            tmem_wait_ld();
-            if (mine && (write_out || !isP)) {  // (P only where outputs are written)
+        for (int kp = 0; kp < 4; kp += 2) {
+          if (kp > a) break;
+          uint32_t v[2][16];
+          tmem_ld16(tl + tm_ap + ap_off(a) + 16 * kp, v[0]);
+          if (kp + 1 <= a) tmem_ld16(tl + tm_ap + ap_off(a) + 16 * (kp + 1), v[1]);
+          tmem_wait_ld();
+          if (mine && (write_out || !isP)) {  // (P only where outputs are written)
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int kb = kp + h2;
+              if (kb > a) break;
               if (!isP) {
 #pragma unroll
-                for (int jj = 0; jj < 16; ++jj) {
-                  const int s = 16 * kb + jj;
-                  Af[t * LDF + s] = (s < t) ? bt * __uint_as_float(v[jj]) : 0.f;
+                for (int c4 = 0; c4 < 4; ++c4) {
+                  const int s = 16 * kb + 4 * c4;
+                  const uint32_t* w = &v[h2][4 * c4];
+                  *reinterpret_cast<float4*>(&Af[t * LDF + s]) = make_float4(
+                      s < t ? bt * __uint_as_float(w[0]) : 0.f, s + 1 < t ? bt * __uint_as_float(w[1]) : 0.f,
+                      s + 2 < t ? bt * __uint_as_float(w[2]) : 0.f, s + 3 < t ? bt * __uint_as_float(w[3]) : 0.f);
                 }
               } else {
 #pragma unroll
                 for (int oc = 0; oc < 2; ++oc) {
                   float f[8];
 #pragma unroll
-                  for (int e = 0; e < 8; ++e) f[e] = (16 * kb + 8 * oc + e <= t) ? __uint_as_float(v[8 * oc + e]) : 0.f;
+                  for (int e = 0; e < 8; ++e)
+                    f[e] = (16 * kb + 8 * oc + e <= t) ? __uint_as_float(v[h2][8 * oc + e]) : 0.f;
                   at16(sm, OFF_P + sw128_oct(t, 2 * kb + oc, 8192)) = pack8(f);
                 }
               }
@@ -920,11 +930,28 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
           else state_copy(warp < 4 ? 0 : 1, warp < 4 ? 1 : 2, snap);
         }
         sync_wg();
+        // T' = T Diag(beta) in bf16, item idx = row i, column octet oc (T is zero above the diagonal)
+        auto pack_tp = [&](int idx) {
+          const int i = idx >> 3, oc = idx & 7;
+          const float4 t0 = *reinterpret_cast<const float4*>(Tf + i * LDT + 8 * oc);
+          const float4 t1 = *reinterpret_cast<const float4*>(Tf + i * LDT + 8 * oc + 4);
+          const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+          float f[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int jc = 8 * oc + e;
+            f[e] = (jc <= i) ? tv[e] * beta[jc] : 0.f;
+          }
+          at16(sm, OFF_TP + sw128_oct(i, oc, 8192)) = pack8(f);
+        };
         // Off-diagonal blocks level by level (block distance d), one 16x8 strip per warp: warp
         // w < 2 (4 - d) takes a = b + d with b = w / 2 and columns 16 b + 8 (w % 2) .. +7:
         //   Y = sum_{c=b}^{a-1} L_ac T_cb,   T_ab = -T_aa Y,
         // as m16n8k8 tf32 MMAs.  Y never leaves the warp: its C fragment becomes the B fragment
-        // of the second product by shuffles.  A level reads only blocks of earlier levels.
+        // of the second product by shuffles.  A level reads only blocks of earlier levels.  The
+        // warps a level leaves idle pack the row blocks of T' that are final: rows 0-15 (final
+        // after the diagonal blocks) beside level 1, rows 16-31 beside level 2, rows 32-47 beside
+        // level 3; rows 48-63 follow the last level.
         {
           const int g = lane >> 2, t4 = lane & 3;
 #pragma unroll
@@ -978,25 +1005,18 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
               float* to = Tf + (16 * a + g) * LDT + 16 * b + n0 + 2 * t4;
               *reinterpret_cast<float2*>(to) = make_float2(o4[0], o4[1]);
               *reinterpret_cast<float2*>(to + 8 * LDT) = make_float2(o4[2], o4[3]);
+            } else if (d == 1) {  // warps 6-7: rows 0-15 (items 0-127)
+              pack_tp(tid - 192);
+              pack_tp(tid - 192 + 64);
+            } else if (d == 2) {  // warps 4-7: rows 16-31 (items 128-255)
+              pack_tp(tid);
+            } else {  // warps 2-7: rows 32-47 (items 256-383), one per thread of warps 2-5
+              if (tid < 192) pack_tp(tid + 192);
             }
             sync_wg();
           }
         }
-#pragma unroll
-        for (int it = 0; it < 2; ++it) {
-          const int idx = tid + kCompute * it;
-          const int i = idx >> 3, oc = idx & 7;
-          const float4 t0 = *reinterpret_cast<const float4*>(Tf + i * LDT + 8 * oc);
-          const float4 t1 = *reinterpret_cast<const float4*>(Tf + i * LDT + 8 * oc + 4);
-          const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-          float f[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int jc = 8 * oc + e;
-            f[e] = (jc <= i) ? tv[e] * beta[jc] : 0.f;
-          }
-          at16(sm, OFF_TP + sw128_oct(i, oc, 8192)) = pack8(f);
-        }
+        if (tid < 128) pack_tp(384 + tid);  // rows 48-63
       }
       // A partial last chunk: the v tile's rows t >= L hold the next sequence's tokens (or the
       // zero fill past the tensor).  T' has zero columns there (beta = 0), but 0 * Inf or NaN is
@@ -1133,13 +1153,7 @@ __device__ __forceinline__ void chunk_tc_body(const Plan& plan, const TcMaps& ma
     // ---------------------------------------------------------------- end state
     if (ok) {
       float* dst = nullptr;
-      if (seg.role == kRoleWhole || seg.role == kRoleFromWs) {
-        if (seg.last) {
-          if (p.final_state) dst = p.final_state + ((size_t)seg.seq * H + h) * unit_state;
-        } else if (seg.role == kRoleWhole) {  // first segment of a split sequence: the next one's start
-          dst = p.ws_state + ((size_t)(seg.slot + 1) * H + h) * unit_state;
-        }
-      }
+      if (kOut && seg.last && p.final_state) dst = p.final_state + ((size_t)seg.seq * H + h) * unit_state;
       size_t ld = DV;
       if (!kOut) {  // pass 1: the (S_loc | M) block of the slot, row stride dv + dk
         ld = DV + DK;

@@ -54,6 +54,11 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
       "l"(*reinterpret_cast<const uint64_t*>(&b)), "l"(*reinterpret_cast<const uint64_t*>(&c)));
   return *reinterpret_cast<const float2*>(&r);
 }
+// Two consecutive outputs (4-byte store for bf16, 8-byte for fp32; c is even)
+__device__ __forceinline__ void store2(__nv_bfloat16* p, float a, float b) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(a, b);
+}
+__device__ __forceinline__ void store2(float* p, float a, float b) { *reinterpret_cast<float2*>(p) = make_float2(a, b); }
 __device__ __forceinline__ float2 lo2(const float4& v) { return make_float2(v.x, v.y); }
 __device__ __forceinline__ float2 hi2(const float4& v) { return make_float2(v.z, v.w); }
 
@@ -268,6 +273,7 @@ struct MultiSmem {
   float sdot[KG][KG][2];          // [j][i]: raw c_ji (i < j), raw d_ji (i <= j)
   float snrm[KG][2];              // |k_j|^2, |q_j|^2
   float sbeta[KG];
+  float sss[KG][DV / 32];         // per warp of the column solve: sum of o_j^2 over its 32 columns
 };
 
 template <typename T, int DK, int DV, bool kPre>
@@ -296,9 +302,11 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const DecodeP
     if (tid == 0) report_error(p.error_word, KDA_ERR_BAD_STATE_INDEX);
     return;
   }
-  // the token inputs of the group starting at `base`: 16-byte cp.async chunks, then beta
+  // the token inputs of the group starting at `base`: 16-byte cp.async chunks, then beta (kept
+  // in its input type until the group's inputs are waited for, so that no thread stalls on it
+  // before the loads behind it are issued)
   constexpr int CK = DK * (int)sizeof(T) / 16, CV = DV * (int)sizeof(T) / 16;  // chunks per row
-  float beta_reg = 0.f;
+  T beta_raw = T();
   auto fetch_group = [&](int base) {
     const int Kg = min(KG, K - base);
     for (int idx = tid; idx < Kg * (3 * CK + 2 * CV); idx += kThreads) {
@@ -323,10 +331,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const DecodeP
       cp_async_16(smem_u32(dst + 16 * c), reinterpret_cast<const uint8_t*>(src) + 16 * c);
     }
     cp_async_commit();
-    if (tid < Kg) beta_reg = to_f32(static_cast<const T*>(p.beta)[((size_t)n * K + base + tid) * p.H + h]);
+    if (tid < Kg) beta_raw = static_cast<const T*>(p.beta)[((size_t)n * K + base + tid) * p.H + h];
   };
-  fetch_group(0);
 
+  // the state first (the longest wait), then the first group's inputs
   float* S = p.state + ((size_t)slot * p.H + h) * (size_t)(DK * DV);
   const int cg = tid % TPR;   // column group: columns 4cg .. 4cg+3
   const int r0 = tid / TPR;   // first row; rows r0 + RPP * i
@@ -334,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const DecodeP
 #pragma unroll
   for (int i = 0; i < NP; ++i)
     s[i] = __ldcs(reinterpret_cast<const float4*>(S + (size_t)(r0 + RPP * i) * DV) + cg);
+  fetch_group(0);
   if (tid == 0 && p.ahead > 0 && unit + p.ahead < (int)gridDim.x) {  // see decode_kernel
     const int u2 = unit + p.ahead;
     const int n2 = u2 / p.H;
@@ -351,7 +360,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const DecodeP
       fetch_group(base);
     }
     cp_async_wait_all();
-    if (tid < Kg) sm.sbeta[tid] = b_logits ? 1.f / (1.f + __expf(-beta_reg)) : beta_reg;  // beta = sigmoid(b)
+    if (tid < Kg) {
+      const float beta = to_f32(beta_raw);
+      sm.sbeta[tid] = b_logits ? 1.f / (1.f + __expf(-beta)) : beta;  // beta = sigmoid(b)
+    }
     __syncthreads();
     // ---- per channel: G_j (prefix over the group), e^{g_j}, and the decayed k, q
     if (tid < DK) {
@@ -477,7 +489,14 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const DecodeP
         u[j] = sm.sbeta[j] * (to_f32(sm.rv[j][tid]) - pred);
         o += sm.sdot[j][j][1] * rqj * rkj * u[j];
         sm.su[j][tid] = u[j];
-        sm.red[0][2 * j][tid] = p.scale * o;
+        const float os = p.scale * o;
+        sm.red[0][2 * j][tid] = os;
+        if (p.gate != nullptr) {  // the RMSNorm's sum of squares, by warp (read after the next barrier)
+          float sq = os * os;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+          if (lane == 0) sm.sss[j][warp] = sq;
+        }
       }
     }
     const bool closed = p.position_states == nullptr;  // only the end state is needed
@@ -539,29 +558,23 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const DecodeP
         for (int i = 0; i < NP; ++i) __stcs(reinterpret_cast<float4*>(P + (size_t)(r0 + RPP * i) * DV) + cg, s[i]);
       }
     }
-    // ---- outputs: warp j takes token j (head-wise RMSNorm over dv, then the sigmoid gate)
-    if (warp < Kg) {
-      const int j = warp;
+    // ---- outputs: column pairs of every token of the group over all threads (head-wise RMSNorm
+    // over dv from the sums of squares of the solve, then the sigmoid gate)
+    for (int idx = tid; idx < Kg * (DV / 2); idx += kThreads) {
+      const int j = idx / (DV / 2), c = 2 * (idx - j * (DV / 2));
       const size_t row = ((size_t)n * K + base + j) * p.H + h;
-      T* op = static_cast<T*>(p.out) + row * DV;
-      const float* so = sm.red[0][2 * j];
-      if (p.gate == nullptr) {
-#pragma unroll
-        for (int c = lane; c < DV; c += 32) op[c] = from_f32<T>(so[c]);
-      } else {
+      T* op = static_cast<T*>(p.out) + row * DV + c;
+      float y0 = sm.red[0][2 * j][c], y1 = sm.red[0][2 * j][c + 1];
+      if (p.gate != nullptr) {
         float ss = 0.f;
 #pragma unroll
-        for (int c = lane; c < DV; c += 32) ss += so[c] * so[c];
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        for (int w = 0; w < DV / 32; ++w) ss += sm.sss[j][w];
         const float rr = rsqrtf(ss / (float)DV + p.eps);
-#pragma unroll
-        for (int c = lane; c < DV; c += 32) {
-          const float wj = p.norm_weight ? p.norm_weight[c] : 1.0f;
-          const float gl = to_f32(sm.rgate[j][c]);
-          op[c] = from_f32<T>(so[c] * rr * wj / (1.0f + __expf(-gl)));
-        }
+        const float w0 = p.norm_weight ? p.norm_weight[c] : 1.0f, w1 = p.norm_weight ? p.norm_weight[c + 1] : 1.0f;
+        y0 *= rr * w0 / (1.0f + __expf(-to_f32(sm.rgate[j][c])));
+        y1 *= rr * w1 / (1.0f + __expf(-to_f32(sm.rgate[j][c + 1])));
       }
+      store2(op, y0, y1);
     }
   }
 }

@@ -19,9 +19,8 @@ constexpr int kPlanMax = 960;  // segments per launch (the plan travels in the k
 
 // Where a unit's start state comes from and where its end state goes.
 enum SegRole : int32_t {
-  kRoleWhole = 0,     // start: initial_state (or 0); writes outputs; end: final_state if the segment
-                      //   ends its sequence, else (the first segment of a split sequence) the
-                      //   workspace start-state slot of the next segment
+  kRoleWhole = 0,     // an unsplit sequence: start: initial_state (or 0); writes outputs;
+                      //   end: final_state
   kRoleLocal = 1,     // split pass 1: start from [0 | I] (the augmented state [S | M], values
                       //   augmented by zeros), no outputs; end: workspace slot (S_loc | M)
   kRoleFromWs = 3,    // split pass 2: start from workspace start-state slot; writes outputs;

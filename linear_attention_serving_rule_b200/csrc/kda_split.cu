@@ -8,11 +8,12 @@
 //     S_end(q) = M_q S_start(q) + S_loc(q)
 //
 // where pass 1 computed (S_loc(q) | M_q) by running the segment from [0 | I] with values
-// augmented by zeros.  This kernel chains the segments:
+// augmented by zeros.  This kernel chains the segments from the sequence's initial state:
 //
-//     S_start(q+1) = M_q S_start(q) + S_loc(q),   q = 1 .. nseg-2
+//     S_start(0) = S_init (zero without one),   S_start(q+1) = M_q S_start(q) + S_loc(q),
+//     q = 0 .. nseg-2,
 //
-// (S_start(1) was written by the head segment, which ran from the true initial state).
+// and leaves every S_start(q) in the workspace for the pass that writes the outputs.
 // Value columns are independent, so each CTA owns a block of 16 state columns of one
 // (sequence, head) and walks the segments in order.
 #include "kda_internal.cuh"
@@ -40,11 +41,17 @@ __global__ void __launch_bounds__(kThreads) combine_kernel(const __grid_constant
   constexpr int NR = DK / RS;           // rows per thread
 
   const size_t unit = (size_t)DK * DV;
-  float* st = p.ws_state + ((size_t)(b + 1) * H + h) * unit;
+  const float* init = p.initial_state ? p.initial_state + ((size_t)s.seq * H + h) * unit : nullptr;
+  float* st = p.ws_state + ((size_t)b * H + h) * unit;
 #pragma unroll
-  for (int r = 0; r < NR; ++r) sc[i0 + RS * r][j] = st[(size_t)(i0 + RS * r) * DV + j0 + j];
+  for (int r = 0; r < NR; ++r) {
+    const size_t e = (size_t)(i0 + RS * r) * DV + j0 + j;
+    const float x = init ? init[e] : 0.f;
+    sc[i0 + RS * r][j] = x;
+    st[e] = x;
+  }
   __syncthreads();
-  for (int q = 1; q <= nseg - 2; ++q) {
+  for (int q = 0; q <= nseg - 2; ++q) {
     const float* loc = p.ws_local + ((size_t)(b + q) * H + h) * (size_t)DK * LD;
     float acc[NR];
 #pragma unroll

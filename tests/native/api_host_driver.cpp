@@ -97,18 +97,26 @@ void run_and_check(kda_chunk_args a, const std::vector<int32_t>& lens, bool expe
   bool any_split = false;
   int combine_units = 0;
   std::map<int, int> pass1;  // slot -> count of pass-1 results
+  int stage = 0;  // 0: pass 1, 1: combine, 2: outputs; launches never go back a stage
   for (const Launch& L : g_launches) {
     CHECK(L.kind == 't' || L.kind == 's' || L.kind == 'c');
     CHECK(L.H == a.H);
     CHECK(!L.segs.empty() && (int)L.segs.size() <= kda::kPlanMax);
     if (L.kind == 'c') {
+      CHECK(stage <= 1);
+      stage = 1;
       for (const auto& s : L.segs) {
-        CHECK(s.len >= 3 && s.slot >= 0);  // the segment count travels in len
+        CHECK(s.len >= 2 && s.slot >= 0);  // the segment count travels in len
         combine_units += 1;
       }
       continue;
     }
     for (size_t i = 1; i < L.segs.size(); ++i) CHECK(L.segs[i - 1].len >= L.segs[i].len);  // longest first
+    // one kind of unit per launch: pass 1 only, or output units only
+    const bool is_pass1 = L.segs[0].role == kda::kRoleLocal;
+    for (const auto& s : L.segs) CHECK((s.role == kda::kRoleLocal) == is_pass1);
+    CHECK(is_pass1 ? stage == 0 : true);
+    if (!is_pass1) stage = 2;
     for (const auto& s : L.segs) {
       CHECK(s.seq >= 0 && s.seq < N);
       // an empty unit only for an empty sequence (it copies the initial state to the final one)
@@ -139,11 +147,15 @@ void run_and_check(kda_chunk_args a, const std::vector<int32_t>& lens, bool expe
       at += v[i].len;
       CHECK(v[i].last == (i + 1 == v.size() ? 1 : 0));
       if (i + 1 < v.size()) CHECK(v[i].len % 64 == 0);
-      CHECK(v[i].role == (i == 0 ? kda::kRoleWhole : kda::kRoleFromWs));
+      // an unsplit sequence runs whole from its initial state; every segment of a split one from
+      // the start state the combine left in its slot, and all but the last also ran pass 1
+      CHECK(v[i].role == (v.size() == 1 ? kda::kRoleWhole : kda::kRoleFromWs));
+      if (v.size() > 1) CHECK(pass1.count(v[i].slot) == (i + 1 < v.size() ? 1u : 0u));
     }
     CHECK(at == tok0[n + 1]);
   }
-  (void)combine_units;
+  for (const auto& kv : pass1) CHECK(kv.second == 1);
+  CHECK(any_split == (combine_units > 0));  // a split sequence always needs its start states chained
 }
 
 int main() {

@@ -138,13 +138,13 @@ def test_workspace_size_and_check(L):
 
 def test_automatic_split_for_long_context(L):
     # 1 sequence x 16 heads of 1M tokens: 16 units < half of 148 SMs -> split.  With P segments
-    # the first launch holds 16 x (1 + 2 (P - 2)) units (each first segment in full, S_loc and M
-    # of each middle one) and the last 16 x (P - 1); P = 10 gives 272 units (2 waves of 148) and
-    # 144 (1 wave): 3/10 of the unsplit time, the least for P <= 64.
+    # the first launch holds 16 x (P - 1) units (pass 1 of every segment but the last) and the
+    # second 16 x P (every segment with its outputs); P = 9 gives 128 and 144 units, one wave of
+    # 148 each: 2/9 of the unsplit time, the least for P <= 64 (P = 18 ties at 4 waves / 18).
     rc, n = _ws(L, _args(num_seqs=1, total_tokens=1 << 20, H=16))
     assert rc == B.KDA_OK
     per_slot = 16 * (128 * 128 + 128 * 256) * 4
-    assert (n - 256) % per_slot == 0 and (n - 256) // per_slot == 10
+    assert (n - 256) % per_slot == 0 and (n - 256) // per_slot == 9
 
 
 def _dargs(**kw):
