@@ -126,6 +126,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     const T* kp = static_cast<const T*>(p.k) + row * DK;
     const T* qp = static_cast<const T*>(p.q) + row * DK;
     const T* gp = static_cast<const T*>(p.g) + row * DK;
+    // the token's other inputs are issued now, with k, q and g, and kept in their input type until
+    // they are used, so that none of them is a memory round trip of its own later in the step
+    T v_raw = T(), gate_raw = T(), beta_raw = T();
+    float w_norm = 1.f;
+    if (tid < DV) {
+      v_raw = static_cast<const T*>(p.v)[row * DV + tid];
+      if (p.gate != nullptr) gate_raw = static_cast<const T*>(p.gate)[row * DV + tid];
+      if (p.norm_weight) w_norm = p.norm_weight[tid];
+    }
+    beta_raw = static_cast<const T*>(p.beta)[row];
     for (int i = tid; i < DK; i += kThreads) {
       sk[i] = to_f32(kp[i]);
       sq[i] = to_f32(qp[i]);
@@ -177,17 +187,23 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     reinterpret_cast<float4*>(red_q[r0])[cg] = yq;
     __syncthreads();
 
-    float beta = to_f32(static_cast<const T*>(p.beta)[row]);
+    float beta = to_f32(beta_raw);
     if (kPre && (p.flags & KDA_FLAG_BETA_LOGITS)) beta = 1.f / (1.f + expf(-beta));  // beta = sigmoid(b)
     const float rk = kPre ? s_rk : 1.f;
     if (tid < DV) {
       float ak = 0.f, aq = 0.f;
   #pragma unroll
       for (int r = 0; r < RPP; ++r) { ak += red_k[r][tid]; aq += red_q[r][tid]; }
-      const float vj = to_f32(static_cast<const T*>(p.v)[row * DV + tid]);
-      const float u = beta * (vj - ak * rk);
+      const float u = beta * (to_f32(v_raw) - ak * rk);
       su[tid] = u;
-      so[tid] = p.scale * (kPre ? aq * s_rq + u * s_kq : aq + u * s_kq);
+      const float o = p.scale * (kPre ? aq * s_rq + u * s_kq : aq + u * s_kq);
+      so[tid] = o;
+      if (p.gate != nullptr) {  // the RMSNorm's sum of squares, by warp (read after the next barrier)
+        float ss = o * o;
+  #pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        if ((tid & 31) == 0) s_ss[tid >> 5] = ss;
+      }
     }
     __syncthreads();
 
@@ -206,29 +222,18 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams 
     }
 
     T* op = static_cast<T*>(p.out) + row * DV;
-    if (p.gate == nullptr) {
-      if (tid < DV) op[tid] = from_f32<T>(so[tid]);
-      continue;
-    }
-    // head-wise RMSNorm over dv, then the sigmoid gate
-    float o = 0.f;
     if (tid < DV) {
-      o = so[tid];
-      float ss = o * o;
+      const float o = so[tid];
+      if (p.gate == nullptr) {
+        op[tid] = from_f32<T>(o);
+      } else {  // head-wise RMSNorm over dv (the sums of squares from the solve), then the sigmoid gate
+        float tot = 0.f;
   #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-      if ((tid & 31) == 0) s_ss[tid >> 5] = ss;
-    }
-    __syncthreads();
-    if (tid < DV) {
-      float tot = 0.f;
-  #pragma unroll
-      for (int w = 0; w < DV / 32; ++w) tot += s_ss[w];
-      const float r = rsqrtf(tot / (float)DV + p.eps);
-      const float wj = p.norm_weight ? p.norm_weight[tid] : 1.0f;
-      const float gl = to_f32(static_cast<const T*>(p.gate)[row * DV + tid]);
-      const float sig = 1.0f / (1.0f + expf(-gl));
-      op[tid] = from_f32<T>(o * r * wj * sig);
+        for (int w = 0; w < DV / 32; ++w) tot += s_ss[w];
+        const float r = rsqrtf(tot / (float)DV + p.eps);
+        const float sig = 1.0f / (1.0f + expf(-to_f32(gate_raw)));
+        op[tid] = from_f32<T>(o * r * w_norm * sig);
+      }
     }
   }
 }
