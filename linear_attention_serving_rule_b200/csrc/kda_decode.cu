@@ -301,6 +301,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const DecodeP
   const bool l2norm = kPre && (p.flags & KDA_FLAG_QK_L2NORM) != 0;
   const bool b_logits = kPre && (p.flags & KDA_FLAG_BETA_LOGITS) != 0;
   const int K = p.tokens;
+  const bool closed = p.position_states == nullptr;  // only the end state is needed
 
   int slot = p.state_indices ? p.state_indices[n] : n;
   if (slot < 0 || slot >= p.num_slots) {  // uniform over the block
@@ -381,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const DecodeP
           report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
         sm.sk[j][tid] = kx;
         sm.sq[j][tid] = qx;
-        sm.sa[j][tid] = __expf(gi);
+        if (!closed) sm.sa[j][tid] = __expf(gi);  // (only the token-by-token update reads it)
         acc += gi;
         sm.sg[j][tid] = acc;
         const float e = __expf(acc);
@@ -504,13 +505,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const DecodeP
         }
       }
     }
-    const bool closed = p.position_states == nullptr;  // only the end state is needed
-    if (closed && tid < DK) {
-      const float gl = sm.sg[Kg - 1][tid];
-      sm.wK[tid] = __expf(gl);
+    // the end state's factors, on the last DK threads: beside the column solve of the first DV
+    static_assert(DK + DV <= kThreads, "the factor threads follow the solve threads");
+    if (closed && tid >= kThreads - DK) {
+      const int c = tid - (kThreads - DK);
+      const float gl = sm.sg[Kg - 1][c];
+      sm.wK[c] = __expf(gl);
       for (int j = 0; j < Kg; ++j) {
         const float rkj = l2norm ? rsqrtf(sm.snrm[j][0] + KDA_L2NORM_EPS) : 1.f;
-        sm.wk[j][tid] = __expf(gl - sm.sg[j][tid]) * sm.sk[j][tid] * rkj;
+        sm.wk[j][c] = __expf(gl - sm.sg[j][c]) * sm.sk[j][c] * rkj;
       }
     }
     __syncthreads();
