@@ -371,24 +371,34 @@ __global__ void __launch_bounds__(kThreads, 2) decode_multi_kernel(const DecodeP
       sm.sbeta[tid] = b_logits ? 1.f / (1.f + __expf(-beta)) : beta;  // beta = sigmoid(b)
     }
     __syncthreads();
-    // ---- per channel: G_j (prefix over the group), e^{g_j}, and the decayed k, q
-    if (tid < DK) {
-      float acc = 0.f;
-      for (int j = 0; j < Kg; ++j) {
-        const float kx = to_f32(sm.rk[j][tid]), qx = to_f32(sm.rq[j][tid]);
-        float gi = to_f32(sm.rg[j][tid]);
+    // ---- per channel: G_j (prefix over the group), e^{g_j}, and the decayed k, q.  Every thread
+    // takes one channel and a run of TPP tokens; it first sums the decay of the tokens before its
+    // run, in the same order as the thread of the run before, so G_j is the same value either way.
+    {
+      constexpr int NPART = kThreads / DK;            // threads per channel
+      constexpr int TPP = (KG + NPART - 1) / NPART;   // tokens per thread
+      const int c = tid % DK, j0 = (tid / DK) * TPP;
+      auto decay = [&](int j) {
+        float gi = to_f32(sm.rg[j][c]);
         if (g_logits) gi = KDA_G_MIN / (1.f + __expf(-gi));  // g = g_min sigmoid(a)
+        return gi;
+      };
+      float acc = 0.f;
+      for (int j = 0; j < j0 && j < Kg; ++j) acc += decay(j);
+      for (int j = j0; j < j0 + TPP && j < Kg; ++j) {
+        const float kx = to_f32(sm.rk[j][c]), qx = to_f32(sm.rq[j][c]);
+        const float gi = decay(j);
         if (checked && !(((p.flags & KDA_FLAG_UNBOUNDED_DECAY) || gi >= KDA_G_MIN) && gi <= 0.0f))
           report_error(p.error_word, KDA_ERR_DECAY_OUT_OF_RANGE);
-        sm.sk[j][tid] = kx;
-        sm.sq[j][tid] = qx;
-        if (!closed) sm.sa[j][tid] = __expf(gi);  // (only the token-by-token update reads it)
+        sm.sk[j][c] = kx;
+        sm.sq[j][c] = qx;
+        if (!closed) sm.sa[j][c] = __expf(gi);  // (only the token-by-token update reads it)
         acc += gi;
-        sm.sg[j][tid] = acc;
+        sm.sg[j][c] = acc;
         const float e = __expf(acc);
-        sm.skg[j][tid] = kx * e;
-        sm.sqg[j][tid] = qx * e;
-        sm.ski[j][tid] = kx * __expf(-acc);
+        sm.skg[j][c] = kx * e;
+        sm.sqg[j][c] = qx * e;
+        sm.ski[j][c] = kx * __expf(-acc);
       }
     }
     __syncthreads();
