@@ -56,9 +56,12 @@ def _run(t, state, idx=None, flags=0, pos=None):
                                state_indices=idx, flags=flags, position_states=pos)
 
 
-@pytest.mark.parametrize("K", [1, 2, 4, 8])
-@pytest.mark.parametrize("dtype,dk,dv", [("bf16", 128, 128), ("f32", 64, 128), ("bf16", 128, 64)])
+@pytest.mark.parametrize("K", [1, 2, 3, 4, 5, 7, 8])
+@pytest.mark.parametrize("dtype,dk,dv", [("bf16", 128, 128), ("f32", 64, 128), ("bf16", 128, 64), ("bf16", 64, 64)])
 def test_multi_token_matches_sequential_steps(K, dtype, dk, dv):
+    """K tokens in groups of up to four: K = 3 leaves a partial first group, K = 5 and 7 a partial
+    second group (one and three tokens), so every split of a group's tokens over the threads of
+    a channel is reached."""
     N, H, slots = 5, 3, 9
     state = synth.make_states(slots=slots, H=H, dk=dk, dv=dv, seed=60, device="cuda")
     idx = torch.tensor([8, 0, 3, 6, 1], dtype=torch.int32, device="cuda")
