@@ -147,6 +147,26 @@ def test_automatic_split_for_long_context(L):
     assert (n - 256) % per_slot == 0 and (n - 256) // per_slot == 9
 
 
+@pytest.mark.parametrize("H,T,P", [(8, 1 << 20, 18), (4, 1 << 20, 37), (32, 1 << 16, 9), (64, 1 << 20, 1)])
+def test_automatic_split_segment_count(L, H, T, P):
+    """The planner's model, in chunk times of one unit: waves(H (P - 1)) + waves(H P) launches of a
+    segment's chunks plus 4 per combine step, against the unsplit T / 64.
+    - H = 8, 2^20 tokens: P = 18 gives 136 and 144 units (one wave each): 2 x 911 + 68 = 1,890.
+      P = 37 gives 288 and 296 units (two waves each): 4 x 443 + 144 = 1,916.
+    - H = 4: P = 37 gives 144 and 148 units, 2 x 443 + 144 = 1,030.
+    - H = 32, 2^16 tokens: P = 9 gives 256 and 288 units (two waves each): 4 x 114 + 32 = 488.
+      P = 4 gives 96 and 128 units: 2 x 256 + 12 = 524.
+    - H = 64: no count saves a fifth of 16,384 (P = 2 already takes 2 x 8,192 + 4), so there is no
+      split."""
+    rc, n = _ws(L, _args(num_seqs=1, total_tokens=T, H=H))
+    assert rc == B.KDA_OK
+    per_slot = H * (128 * 128 + 128 * 256) * 4
+    if P == 1:
+        assert n == 256
+    else:
+        assert (n - 256) % per_slot == 0 and (n - 256) // per_slot == P
+
+
 def _dargs(**kw):
     a = B.KdaDecodeArgs()
     a.N, a.H, a.dk, a.dv, a.dtype = 8, 4, 128, 128, B.KDA_BF16
