@@ -158,3 +158,22 @@ def test_multi_token_full_size():
     o_ref, _ = _oracle_steps(t, s64, None)
     assert rel_l2(host(out), o_ref) <= TOL_OUT_BF16
     assert rel_l2(state.cpu().numpy(), s64) <= TOL_STATE_BF16
+
+
+def test_multi_token_bad_state_index_reports_error():
+    """A slot outside the pool is reported on the error word and skipped: no other slot changes,
+    and the valid sequence is still decoded."""
+    N, H, K, slots = 2, 2, 3, 4
+    state = synth.make_states(slots=slots, H=H, dk=128, dv=128, seed=71, device="cuda")
+    before = state.clone()
+    t = _tokens(N, K, H, 128, 128, "bf16", seed=72)
+    idx = torch.tensor([1, 4], dtype=torch.int32, device="cuda")  # 4 is out of range
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kda.kda_decode_step(t["q"], t["k"], t["v"], t["g"], t["beta"], state, gate=t["gate"],
+                        state_indices=idx, error_word=err)
+    assert kda.kda_read_device_error(err) == kda.binding.KDA_ERR_BAD_STATE_INDEX
+    assert torch.equal(state[[0, 2, 3]], before[[0, 2, 3]])  # only slot 1 was touched
+    s64 = before.double().cpu().numpy()
+    one = {n: x[:1].contiguous() for n, x in t.items()}
+    _oracle_steps(one, s64, torch.tensor([1], dtype=torch.int32))
+    assert rel_l2(state[1].cpu().numpy(), s64[1]) <= TOL_STATE_BF16
