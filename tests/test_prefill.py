@@ -52,17 +52,20 @@ def test_tiny_fp32_workload():
     assert rel_l2(host(fin), f_ref) <= TOL_F32
 
 
+@pytest.mark.parametrize("split", [0, 3])
 @pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("dtype,dk,dv", [("bf16", 128, 128), ("f32", 128, 128), ("bf16", 64, 128),
                                          ("f32", 64, 64), ("bf16", 128, 64)])
-def test_ragged_varlen_small(path, dtype, dk, dv):
+def test_ragged_varlen_small(path, dtype, dk, dv, split):
     """Chunk-boundary edge cases in one packed batch: lengths 0, 1, 15, 16, 17, 63, 64, 65,
-    127, 200 with initial states, gate and a norm weight; every element compared."""
+    127, 200 with initial states, gate and a norm weight; every element compared.  With a forced
+    split of 3 the sequences longer than one chunk are cut into two segments (64 + 1, 64 + 63,
+    128 + 72) while the others run whole beside them, the empty one included."""
     lengths = np.array([1, 15, 0, 16, 17, 63, 64, 65, 127, 200])
     inp = synth.make_prefill(H=3, dk=dk, dv=dv, dtype=dtype, seed=31, device="cuda",
                              lengths=lengths, gate=True, init_state=True)
     w = torch.linspace(0.5, 1.5, dv, device="cuda")
-    out, fin = _run(inp, flags=PATHS[path], norm_weight=w)
+    out, fin = _run(inp, flags=PATHS[path], norm_weight=w, split=split)
     o_ref, f_ref = oracle_full(inp, norm_weight=w)
     to, ts = _tol(inp)
     assert rel_l2(host(out), o_ref) <= to
