@@ -372,6 +372,23 @@ def pin_scalar_worked_example(ref):
     np.testing.assert_allclose(fin.reshape(-1), [a + b * e], rtol=1e-15)
 
 
+def pin_default_scale_is_one_over_sqrt_dk(ref):
+    """The read-out is o_t = S_t^T q_t / sqrt(dk) when no scale is passed.  Worked by hand: dk = 4,
+    dv = 1, one token with k = q = (1/2, 1/2, 1/2, 1/2) (unit norm), v = 2, g = 0, beta = 1 from
+    S0 = 0.  The write gives S_1 = k v = 2 k, so o = scale * 2 (k . q) = 2 scale = 2 / sqrt(4) = 1,
+    and the decode step gives the same.  (A 1/dk default would give 0.5.)"""
+    half = np.full((1, 1, 4), 0.5, dtype=np.float32)
+    v = np.full((1, 1, 1), 2.0, dtype=np.float32)
+    g = np.zeros((1, 1, 4), dtype=np.float32)
+    beta = np.ones((1, 1), dtype=np.float32)
+    out, fin = ref.forward(half, half, v, g, beta)
+    assert out.reshape(-1).tolist() == [1.0]
+    assert fin.reshape(-1).tolist() == [1.0, 1.0, 1.0, 1.0]
+    state = np.zeros((1, 1, 4, 1))
+    o = ref.decode_step(half, half, v, g, beta, state)
+    assert np.asarray(o).reshape(-1).tolist() == [1.0]
+
+
 # --- I9: the decay floor keeps 16-token factors inside the bf16 range ------------------------
 def pin_decay_floor_bound_on_generated_inputs(ref):
     """g = -5 sigmoid(.) >= -5 after bf16 rounding, so any 16-token cumulative log-decay is
@@ -390,7 +407,8 @@ PINS = [pin_delta_write_is_exact_for_unit_keys, pin_beta_zero_is_pure_decay,
         pin_split_invariance_and_varlen_packing, pin_epilogue_matches_library_rmsnorm,
         pin_decode_step_matches_one_token_forward, pin_scalar_worked_example,
         pin_snapshots_are_unrolled_prefix_states, pin_decay_logits_are_the_scaled_sigmoid,
-        pin_beta_logits_are_the_sigmoid, pin_qk_l2norm_gives_unit_keys]
+        pin_beta_logits_are_the_sigmoid, pin_qk_l2norm_gives_unit_keys,
+        pin_default_scale_is_one_over_sqrt_dk]
 
 
 @pytest.fixture(scope="module")
